@@ -1,0 +1,134 @@
+/*
+ * sink_attn.h - C ABI of libsinkattn.so: causal grouped-query attention with
+ * a learned per-head attention sink, an optional sliding window and optional
+ * packed documents (varlen), forward and backward, for NVIDIA B200 (sm_100a).
+ *
+ * The operation.  Attention sinks are named in "gpt-oss implementation"
+ * (Megatron-LM issue 1739), section "Attention Mechanisms / Attention Sinks"
+ * (after StreamingLLM), in "Tricks from OpenAI gpt-oss you can use with
+ * transformers" ("Flash Attention 3 with support for attention sinks") and
+ * in tpu-inference PR 861 (a kernel argument `attention_sink`).  The pages
+ * name the sink without writing it out; the reading implemented here is the
+ * gpt-oss one: one extra logit s_h per query head joins each row's softmax
+ * denominator and carries no value:
+ *
+ *   l_ij  = scale * q_i . k_j                      (j allowed for row i)
+ *   m_i   = max(s_h, max_j l_ij)
+ *   out_i = sum_j e^{l_ij - m_i} v_j / (e^{s_h - m_i} + sum_j e^{l_ij - m_i})
+ *   lse_i = m_i + ln(e^{s_h - m_i} + sum_j e^{l_ij - m_i})   (sink included)
+ *
+ * s_h is used as given (it is not multiplied by `scale`); s_h = -INFINITY
+ * turns the sink off.  Query head h reads key/value head h / (Hq / Hkv).
+ *
+ * Allowed keys.  Positions are local to a document.  For doc-local query
+ * position i, key j is allowed iff j <= i and, when window > 0, i - j < window
+ * (a window of `window` keys including the query itself).  window <= 0 is
+ * full causal.  The alternating sliding-window / full-causal layer pattern of
+ * "gpt-oss implementation" ("Alternating Sliding-Window Attention Pattern")
+ * is the caller choosing `window` per layer.  Documents follow the
+ * intra-document masking request in the same issue: no attention crosses a
+ * cu_seqlens boundary.
+ *
+ * Backward (derivative of the above; dout given):
+ *   P_ij = e^{l_ij - lse_i}, P_sink,i = e^{s_h - lse_i}, D_i = dout_i . out_i
+ *   dS_ij = P_ij (dout_i . v_j - D_i)
+ *   dq_i = scale sum_j dS_ij k_j, dk_j = scale sum_{i, h in group} dS_ij q_i,
+ *   dv_j = sum_{i, h in group} P_ij dout_i, dsinks_h = -sum_i P_sink,i D_i.
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are DEVICE pointers owned by the caller; the
+ *     library never allocates, frees or synchronises, and every call is
+ *     asynchronous on `stream` (a cudaStream_t passed as void*, NULL = the
+ *     legacy default stream).
+ *   - Arguments are validated on the host before any launch; a failed check
+ *     returns an error status and launches nothing.
+ *   - Layouts are dense and row-major: q/out/dout/dq [T][Hq][D],
+ *     k/v/dk/dv [T][Hkv][D] (bf16), lse [Hq][T] (fp32), sinks/dsinks [Hq]
+ *     (fp32), cu_seqlens [batch+1] (int32, device, cu_seqlens[0] = 0,
+ *     cu_seqlens[batch] = T, non-decreasing).
+ *   - Supported: D = 64; Hq % Hkv == 0 with G = Hq / Hkv a power of two
+ *     <= 128; scale finite and > 0; bf16 tensors 16-byte aligned.
+ *   - A device-side wait that exceeds its time limit (about one second; it
+ *     never happens in a correct build) makes the kernel record an error
+ *     code and return instead of hanging; sink_attn_device_error() reads it.
+ */
+#ifndef SINK_ATTN_H_
+#define SINK_ATTN_H_
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    SINK_ATTN_OK = 0,
+    SINK_ATTN_ERR_NULL = 1,          /* a required pointer is NULL */
+    SINK_ATTN_ERR_SHAPE = 2,         /* inconsistent or negative sizes */
+    SINK_ATTN_ERR_ALIGN = 3,         /* a tensor is not 16-byte aligned */
+    SINK_ATTN_ERR_UNSUPPORTED = 4,   /* valid, but outside what this build implements */
+    SINK_ATTN_ERR_CUDA = 5,          /* a CUDA runtime/driver call failed */
+    SINK_ATTN_ERR_DEVICE_TIMEOUT = 6,/* a kernel gave up on a wait (see sink_attn_device_error) */
+    SINK_ATTN_ERR_WORKSPACE = 7      /* workspace missing or smaller than sink_attn_bwd_workspace_size() */
+} sink_attn_status;
+
+typedef struct {
+    int batch;        /* B: number of documents (cu_seqlens has batch+1 entries) */
+    int max_seqlen;   /* >= every document length; with cu_seqlens == NULL the
+                         common length S of every document (T = B * S) */
+    int total_tokens; /* T */
+    int num_q_heads;  /* Hq */
+    int num_kv_heads; /* Hkv */
+    int head_dim;     /* D (64) */
+} sink_attn_dims;
+
+/* Forward.  q [T][Hq][D] bf16, k, v [T][Hkv][D] bf16, sinks [Hq] fp32 (may
+ * hold -INFINITY), cu_seqlens int32 [batch+1] on the device or NULL (then
+ * every document has length max_seqlen).  Writes out [T][Hq][D] bf16 and
+ * lse [Hq][T] fp32 (natural log, sink included).  T = 0 is a no-op. */
+sink_attn_status sink_attn_fwd(const sink_attn_dims* dims,
+                               const void* q, const void* k, const void* v,
+                               const float* sinks, const int* cu_seqlens,
+                               int window, float scale,
+                               void* out, float* lse, void* stream);
+
+/* Bytes of device workspace sink_attn_bwd() needs for these sizes
+ * (fp32 dq accumulator, per-row D_i, per-block sink partials, padding).
+ * Returns 0 when the sizes are invalid. */
+size_t sink_attn_bwd_workspace_size(const sink_attn_dims* dims);
+
+/* Backward.  Inputs as for the forward plus the forward's saved out and lse
+ * and the upstream gradient dout [T][Hq][D] bf16.  Writes (overwrites, does
+ * not accumulate) dq [T][Hq][D], dk, dv [T][Hkv][D] (bf16) and dsinks [Hq]
+ * (fp32).  dsinks is reduced in a fixed order and is bitwise reproducible
+ * run to run; dq is accumulated with fp32 atomics and may differ in the last
+ * bits between runs.  `workspace` is caller-owned device memory of at least
+ * sink_attn_bwd_workspace_size(dims) bytes, 256-byte aligned; its contents on
+ * entry do not matter. */
+sink_attn_status sink_attn_bwd(const sink_attn_dims* dims,
+                               const void* q, const void* k, const void* v,
+                               const float* sinks, const int* cu_seqlens,
+                               int window, float scale,
+                               const void* out, const float* lse, const void* dout,
+                               void* dq, void* dk, void* dv, float* dsinks,
+                               void* workspace, size_t workspace_bytes,
+                               void* stream);
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* sink_attn_status_string(sink_attn_status s);
+
+/* Synchronises `stream`, then returns and clears the device error code that a
+ * timed-out wait recorded on the current device (0 = none).  This is the only
+ * entry point that synchronises. */
+int sink_attn_device_error(void* stream);
+
+/* Number of kernels one sink_attn_fwd / sink_attn_bwd call launches for
+ * these sizes (0 when T = 0). */
+int sink_attn_fwd_launches(const sink_attn_dims* dims);
+int sink_attn_bwd_launches(const sink_attn_dims* dims);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SINK_ATTN_H_ */

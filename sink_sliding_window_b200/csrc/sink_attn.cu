@@ -1,0 +1,219 @@
+// Host side of libsinkattn.so: argument validation, TMA descriptors and
+// launches for the C ABI declared in include/sink_attn.h.  Everything here is
+// plain host logic; all attention arithmetic runs in the kernels.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "sink_attn.h"
+
+#include "common.cuh"
+#include "fwd_kernel.cuh"
+#include "bwd_kernels.cuh"
+
+namespace sa {
+namespace {
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_tiled() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  return fn;
+}
+
+// 3-D bf16 view [outer][mid][64] of a token-major tensor, 128B swizzle.
+bool make_map_3d(CUtensorMap* map, const void* base, int inner, int mid, int outer, int box_mid, int box_outer) {
+  EncodeTiledFn enc = get_encode_tiled();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(mid),
+                        static_cast<cuuint64_t>(outer)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(inner) * 2, static_cast<cuuint64_t>(inner) * mid * 2};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(inner), static_cast<cuuint32_t>(box_mid),
+                       static_cast<cuuint32_t>(box_outer)};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int ilog2_exact(int x) {
+  if (x <= 0 || (x & (x - 1)) != 0) return -1;
+  int l = 0;
+  while ((1 << l) < x) ++l;
+  return l;
+}
+
+// Validates the sizes and fills the geometry.  T == 0 is valid (no work).
+sink_attn_status check_dims(const sink_attn_dims* d, const int* cu_seqlens, bool packed, int window, float scale,
+                            Geometry* geo) {
+  if (!d) return SINK_ATTN_ERR_NULL;
+  if (d->batch < 0 || d->max_seqlen < 0 || d->total_tokens < 0 || d->num_q_heads <= 0 || d->num_kv_heads <= 0 ||
+      d->head_dim <= 0)
+    return SINK_ATTN_ERR_SHAPE;
+  if (d->num_q_heads % d->num_kv_heads != 0) return SINK_ATTN_ERR_SHAPE;
+  if (!packed && static_cast<int64_t>(d->batch) * d->max_seqlen != d->total_tokens)
+    return SINK_ATTN_ERR_SHAPE;
+  if (d->total_tokens > 0 && d->batch == 0) return SINK_ATTN_ERR_SHAPE;
+  if (d->head_dim != kHeadDim) return SINK_ATTN_ERR_UNSUPPORTED;
+  const int G = d->num_q_heads / d->num_kv_heads;
+  const int gl = ilog2_exact(G);
+  if (gl < 0 || G > kBlockM) return SINK_ATTN_ERR_UNSUPPORTED;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return SINK_ATTN_ERR_UNSUPPORTED;
+  // Token and element indices are formed in 32-bit ints in places.
+  if (static_cast<int64_t>(d->total_tokens) * d->num_q_heads * kHeadDim >= (int64_t(1) << 40) ||
+      d->total_tokens > (1 << 30))
+    return SINK_ATTN_ERR_UNSUPPORTED;
+  geo->T = d->total_tokens;
+  geo->Hq = d->num_q_heads;
+  geo->Hkv = d->num_kv_heads;
+  geo->G_log2 = gl;
+  geo->P_log2 = 7 - gl;
+  geo->num_qblocks = (d->total_tokens + (1 << geo->P_log2) - 1) >> geo->P_log2;
+  geo->batch = d->batch;
+  geo->seqlen = d->max_seqlen;
+  geo->cu_seqlens = cu_seqlens;
+  geo->window = window > 0 ? window : 0;
+  if (!packed && d->total_tokens > 0 && d->max_seqlen <= 0) return SINK_ATTN_ERR_SHAPE;
+  return SINK_ATTN_OK;
+}
+
+template <typename K>
+bool set_smem_once(K kernel, size_t bytes, int* done_flag) {
+  // Per process; the attribute is per function, not per device context.
+  if (*done_flag) return true;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes)) !=
+      cudaSuccess)
+    return false;
+  *done_flag = 1;
+  return true;
+}
+
+}  // namespace
+}  // namespace sa
+
+using namespace sa;
+
+extern "C" {
+
+const char* sink_attn_status_string(sink_attn_status s) {
+  switch (s) {
+    case SINK_ATTN_OK: return "ok";
+    case SINK_ATTN_ERR_NULL: return "a required pointer is NULL";
+    case SINK_ATTN_ERR_SHAPE: return "inconsistent sizes";
+    case SINK_ATTN_ERR_ALIGN: return "a tensor is not 16-byte aligned";
+    case SINK_ATTN_ERR_UNSUPPORTED: return "unsupported configuration (D must be 64, Hq/Hkv a power of two <= 128, scale > 0)";
+    case SINK_ATTN_ERR_CUDA: return "CUDA call failed";
+    case SINK_ATTN_ERR_DEVICE_TIMEOUT: return "a kernel wait timed out";
+    case SINK_ATTN_ERR_WORKSPACE: return "workspace missing or too small";
+  }
+  return "unknown status";
+}
+
+int sink_attn_device_error(void* stream) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return -1;
+  int v = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&v, g_device_error, sizeof(int)) != cudaSuccess) return -1;
+  if (v != 0 && cudaMemcpyToSymbol(g_device_error, &zero, sizeof(int)) != cudaSuccess) return -1;
+  return v;
+}
+
+int sink_attn_fwd_launches(const sink_attn_dims* d) {
+  Geometry geo;
+  if (check_dims(d, nullptr, true, 0, 1.f, &geo) != SINK_ATTN_OK) return 0;
+  return d->total_tokens > 0 ? 1 : 0;
+}
+
+sink_attn_status sink_attn_fwd(const sink_attn_dims* d, const void* q, const void* k, const void* v,
+                               const float* sinks, const int* cu_seqlens, int window, float scale, void* out,
+                               float* lse, void* stream) {
+  Geometry geo;
+  sink_attn_status st = check_dims(d, cu_seqlens, cu_seqlens != nullptr, window, scale, &geo);
+  if (st != SINK_ATTN_OK) return st;
+  if (geo.T == 0) return SINK_ATTN_OK;
+  if (!q || !k || !v || !sinks || !out || !lse) return SINK_ATTN_ERR_NULL;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) ||
+      (reinterpret_cast<uintptr_t>(lse) & 3u) || (reinterpret_cast<uintptr_t>(sinks) & 3u) ||
+      (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u))
+    return SINK_ATTN_ERR_ALIGN;
+
+  const int G = 1 << geo.G_log2;
+  CUtensorMap tq, tk, tv;
+  if (!make_map_3d(&tq, q, kHeadDim, geo.Hq, geo.T, G, 1 << geo.P_log2) ||
+      !make_map_3d(&tk, k, kHeadDim, geo.Hkv, geo.T, 1, kBlockN) ||
+      !make_map_3d(&tv, v, kHeadDim, geo.Hkv, geo.T, 1, kBlockN))
+    return SINK_ATTN_ERR_CUDA;
+
+  static int smem_set = 0;
+  if (!set_smem_once(sink_attn_fwd_kernel, kFwdSmemBytes, &smem_set)) return SINK_ATTN_ERR_CUDA;
+
+  FwdParams p;
+  p.geo = geo;
+  p.scale_log2 = scale * kLog2e;
+  p.sinks = sinks;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.lse = lse;
+  const int64_t grid = static_cast<int64_t>(geo.num_qblocks) * geo.Hkv;
+  if (grid > 0x7fffffff) return SINK_ATTN_ERR_UNSUPPORTED;
+  sink_attn_fwd_kernel<<<static_cast<unsigned>(grid), kFwdThreads, kFwdSmemBytes,
+                         static_cast<cudaStream_t>(stream)>>>(tq, tk, tv, p);
+  return cudaPeekAtLastError() == cudaSuccess ? SINK_ATTN_OK : SINK_ATTN_ERR_CUDA;
+}
+
+size_t sink_attn_bwd_workspace_size(const sink_attn_dims* d) {
+  Geometry geo;
+  if (check_dims(d, nullptr, true, 0, 1.f, &geo) != SINK_ATTN_OK) return 0;
+  return bwd_workspace_layout(geo).total;
+}
+
+int sink_attn_bwd_launches(const sink_attn_dims* d) {
+  Geometry geo;
+  if (check_dims(d, nullptr, true, 0, 1.f, &geo) != SINK_ATTN_OK) return 0;
+  return d->total_tokens > 0 ? kBwdLaunches : 0;
+}
+
+sink_attn_status sink_attn_bwd(const sink_attn_dims* d, const void* q, const void* k, const void* v,
+                               const float* sinks, const int* cu_seqlens, int window, float scale, const void* out,
+                               const float* lse, const void* dout, void* dq, void* dk, void* dv, float* dsinks,
+                               void* workspace, size_t workspace_bytes, void* stream) {
+  Geometry geo;
+  sink_attn_status st = check_dims(d, cu_seqlens, cu_seqlens != nullptr, window, scale, &geo);
+  if (st != SINK_ATTN_OK) return st;
+  if (!dsinks) return SINK_ATTN_ERR_NULL;
+  if (geo.T == 0) {
+    // No rows: every sink gradient is an empty sum.
+    return cudaMemsetAsync(dsinks, 0, sizeof(float) * geo.Hq, static_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? SINK_ATTN_OK
+               : SINK_ATTN_ERR_CUDA;
+  }
+  if (!q || !k || !v || !sinks || !out || !lse || !dout || !dq || !dk || !dv) return SINK_ATTN_ERR_NULL;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(dout) || !aligned16(dq) ||
+      !aligned16(dk) || !aligned16(dv) || (reinterpret_cast<uintptr_t>(lse) & 3u) ||
+      (reinterpret_cast<uintptr_t>(sinks) & 3u) || (reinterpret_cast<uintptr_t>(dsinks) & 3u) ||
+      (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u))
+    return SINK_ATTN_ERR_ALIGN;
+  const BwdWorkspace ws = bwd_workspace_layout(geo);
+  if (!workspace || workspace_bytes < ws.total) return SINK_ATTN_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(workspace) & 255u) return SINK_ATTN_ERR_ALIGN;
+  return bwd_launch(geo, scale, q, k, v, sinks, out, lse, dout, dq, dk, dv, dsinks,
+                    static_cast<uint8_t*>(workspace), ws, static_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"

@@ -1,0 +1,168 @@
+"""ctypes binding of libsinkattn.so (include/sink_attn.h).
+
+Argument marshalling only: shapes and pointers of torch CUDA tensors go in,
+the C-ABI entry points do all the work on the current (or given) stream.
+There is no CPU fallback: if the library is missing, loading raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsinkattn.so")
+_lib = None
+
+STATUS = {
+    0: "SINK_ATTN_OK",
+    1: "SINK_ATTN_ERR_NULL",
+    2: "SINK_ATTN_ERR_SHAPE",
+    3: "SINK_ATTN_ERR_ALIGN",
+    4: "SINK_ATTN_ERR_UNSUPPORTED",
+    5: "SINK_ATTN_ERR_CUDA",
+    6: "SINK_ATTN_ERR_DEVICE_TIMEOUT",
+    7: "SINK_ATTN_ERR_WORKSPACE",
+}
+
+EXPORTS = ("sink_attn_fwd", "sink_attn_bwd", "sink_attn_bwd_workspace_size", "sink_attn_status_string",
+           "sink_attn_device_error", "sink_attn_fwd_launches", "sink_attn_bwd_launches")
+
+
+class SinkAttnError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS.get(status, status)} ({status_string(status)})")
+
+
+class Dims(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int), ("max_seqlen", ctypes.c_int), ("total_tokens", ctypes.c_int),
+                ("num_q_heads", ctypes.c_int), ("num_kv_heads", ctypes.c_int), ("head_dim", ctypes.c_int)]
+
+
+def lib_path() -> str:
+    return _LIB_PATH
+
+
+def load():
+    """Loads libsinkattn.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(_LIB_PATH):
+            raise RuntimeError(f"libsinkattn.so not found at {_LIB_PATH}; build it with "
+                               "`python -m sink_sliding_window_b200.build`")
+        L = ctypes.CDLL(_LIB_PATH)
+        P = ctypes.c_void_p
+        I = ctypes.c_int
+        DP = ctypes.POINTER(Dims)
+        L.sink_attn_fwd.argtypes = [DP, P, P, P, P, P, I, ctypes.c_float, P, P, P]
+        L.sink_attn_fwd.restype = I
+        L.sink_attn_bwd.argtypes = [DP, P, P, P, P, P, I, ctypes.c_float, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]
+        L.sink_attn_bwd.restype = I
+        L.sink_attn_bwd_workspace_size.argtypes = [DP]
+        L.sink_attn_bwd_workspace_size.restype = ctypes.c_size_t
+        L.sink_attn_status_string.argtypes = [I]
+        L.sink_attn_status_string.restype = ctypes.c_char_p
+        L.sink_attn_device_error.argtypes = [P]
+        L.sink_attn_device_error.restype = I
+        L.sink_attn_fwd_launches.argtypes = [DP]
+        L.sink_attn_fwd_launches.restype = I
+        L.sink_attn_bwd_launches.argtypes = [DP]
+        L.sink_attn_bwd_launches.restype = I
+        _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return load().sink_attn_status_string(int(status)).decode()
+
+
+def make_dims(T, Hq, Hkv, D, batch, max_seqlen) -> Dims:
+    return Dims(int(batch), int(max_seqlen), int(T), int(Hq), int(Hkv), int(D))
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_handle(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _geometry(q, k, cu_seqlens, batch, max_seqlen):
+    if q.dim() == 4:  # [B, S, H, D]
+        B, S = q.shape[0], q.shape[1]
+        q = q.reshape(B * S, q.shape[2], q.shape[3])
+        k = k.reshape(B * S, k.shape[2], k.shape[3])
+        batch, max_seqlen = B, S
+    T, Hq, D = q.shape
+    Hkv = k.shape[1]
+    if cu_seqlens is not None:
+        batch = cu_seqlens.numel() - 1
+        if max_seqlen is None:
+            max_seqlen = T
+    if batch is None or max_seqlen is None:
+        raise ValueError("give cu_seqlens, or batch and max_seqlen, or 4-D [B,S,H,D] tensors")
+    return make_dims(T, Hq, Hkv, D, batch, max_seqlen), T, Hq, Hkv, D
+
+
+def fwd(q, k, v, sinks, cu_seqlens=None, window=0, scale=None, *, batch=None, max_seqlen=None, out=None, lse=None,
+        stream=None):
+    """sink_attn_fwd.  q [T,Hq,D] (or [B,S,Hq,D]), k/v [T,Hkv,D] bf16 CUDA;
+    sinks [Hq] fp32; cu_seqlens int32 [B+1] CUDA or None.
+    Returns (out like q, lse [Hq, T] fp32)."""
+    dims, T, Hq, Hkv, D = _geometry(q, k, cu_seqlens, batch, max_seqlen)
+    if scale is None:
+        scale = D ** -0.5
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((Hq, T), dtype=torch.float32, device=q.device)
+    st = load().sink_attn_fwd(ctypes.byref(dims), _ptr(q), _ptr(k), _ptr(v), _ptr(sinks), _ptr(cu_seqlens),
+                              int(window), float(scale), _ptr(out), _ptr(lse), _stream_handle(stream))
+    if st != 0:
+        raise SinkAttnError(st, "sink_attn_fwd")
+    return out, lse
+
+
+def bwd_workspace_size(T, Hq, Hkv, D, batch, max_seqlen) -> int:
+    d = make_dims(T, Hq, Hkv, D, batch, max_seqlen)
+    return int(load().sink_attn_bwd_workspace_size(ctypes.byref(d)))
+
+
+def bwd(q, k, v, sinks, out, lse, dout, cu_seqlens=None, window=0, scale=None, *, batch=None, max_seqlen=None,
+        dq=None, dk=None, dv=None, dsinks=None, workspace=None, stream=None):
+    """sink_attn_bwd.  Returns (dq, dk, dv, dsinks)."""
+    dims, T, Hq, Hkv, D = _geometry(q, k, cu_seqlens, batch, max_seqlen)
+    if scale is None:
+        scale = D ** -0.5
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    dsinks = torch.empty((Hq,), dtype=torch.float32, device=q.device) if dsinks is None else dsinks
+    L = load()
+    need = int(L.sink_attn_bwd_workspace_size(ctypes.byref(dims)))
+    if workspace is None:
+        workspace = torch.empty((max(need, 1),), dtype=torch.uint8, device=q.device)
+    st = L.sink_attn_bwd(ctypes.byref(dims), _ptr(q), _ptr(k), _ptr(v), _ptr(sinks), _ptr(cu_seqlens), int(window),
+                         float(scale), _ptr(out), _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dsinks),
+                         _ptr(workspace), ctypes.c_size_t(workspace.numel()), _stream_handle(stream))
+    if st != 0:
+        raise SinkAttnError(st, "sink_attn_bwd")
+    return dq, dk, dv, dsinks
+
+
+def device_error(stream=None) -> int:
+    return int(load().sink_attn_device_error(_stream_handle(stream)))
+
+
+def fwd_launches(T, Hq, Hkv, D, batch, max_seqlen) -> int:
+    d = make_dims(T, Hq, Hkv, D, batch, max_seqlen)
+    return int(load().sink_attn_fwd_launches(ctypes.byref(d)))
+
+
+def bwd_launches(T, Hq, Hkv, D, batch, max_seqlen) -> int:
+    d = make_dims(T, Hq, Hkv, D, batch, max_seqlen)
+    return int(load().sink_attn_bwd_launches(ctypes.byref(d)))

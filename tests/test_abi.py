@@ -1,0 +1,107 @@
+"""The C-ABI library loads on a machine without a GPU, exports every
+function include/sink_attn.h declares, and rejects bad arguments on the host
+before touching the device.  CPU only: no call here launches a kernel."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from sink_sliding_window_b200 import build, ops
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return ops.load()
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "sink_attn.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(sink_attn_\w+)\s*\(", src)))
+
+
+def test_exports_every_declared_symbol(L):
+    names = declared_functions()
+    assert "sink_attn_fwd" in names and "sink_attn_bwd" in names
+    for n in names:
+        assert hasattr(L, n), f"{n} declared in include/sink_attn.h but not exported"
+    assert set(ops.EXPORTS) <= set(names)
+
+
+def test_status_strings(L):
+    for code in range(8):
+        s = ops.status_string(code)
+        assert isinstance(s, str) and s
+    assert ops.status_string(99) == "unknown status"
+
+
+def dims(**kw):
+    base = dict(T=256, Hq=8, Hkv=2, D=64, batch=2, max_seqlen=128)
+    base.update(kw)
+    return ops.make_dims(base["T"], base["Hq"], base["Hkv"], base["D"], base["batch"], base["max_seqlen"])
+
+
+FAKE = ctypes.c_void_p(1 << 20)  # 16-byte aligned, never dereferenced: validation fails first
+
+
+def call_fwd(L, d, q=FAKE, k=FAKE, v=FAKE, sinks=FAKE, cu=None, window=0, scale=0.125, out=FAKE, lse=FAKE):
+    return L.sink_attn_fwd(ctypes.byref(d), q, k, v, sinks, cu, window, scale, out, lse, None)
+
+
+@pytest.mark.parametrize("bad,code", [
+    (dict(D=128), 4),            # only D = 64
+    (dict(Hq=6, Hkv=4), 2),      # Hq % Hkv != 0
+    (dict(Hq=12, Hkv=4), 4),     # G = 3 is not a power of two
+    (dict(T=255), 2),            # uniform batch: T != B * S
+    (dict(T=-1), 2),
+    (dict(Hkv=0), 2),
+    (dict(batch=0, max_seqlen=0), 2),
+])
+def test_fwd_rejects_bad_shapes(L, bad, code):
+    assert call_fwd(L, dims(**bad)) == code
+
+
+def test_fwd_rejects_null_and_misaligned(L):
+    assert L.sink_attn_fwd(None, FAKE, FAKE, FAKE, FAKE, None, 0, 0.125, FAKE, FAKE, None) == 1
+    assert call_fwd(L, dims(), q=None) == 1
+    assert call_fwd(L, dims(), lse=None) == 1
+    assert call_fwd(L, dims(), k=ctypes.c_void_p((1 << 20) + 8)) == 3
+    assert call_fwd(L, dims(), out=ctypes.c_void_p((1 << 20) + 2)) == 3
+
+
+def test_fwd_rejects_bad_scale(L):
+    for s in (0.0, -0.125, float("inf"), float("nan")):
+        assert call_fwd(L, dims(), scale=s) == 4
+
+
+def test_fwd_empty_is_noop(L):
+    # T = 0: valid, nothing to do, no pointer is touched.
+    assert call_fwd(L, dims(T=0, batch=0, max_seqlen=0), q=None, k=None, v=None, out=None, lse=None) == 0
+
+
+def test_bwd_workspace_and_validation(L):
+    d = dims()
+    ws = L.sink_attn_bwd_workspace_size(ctypes.byref(d))
+    assert ws > 0
+    assert L.sink_attn_bwd_workspace_size(ctypes.byref(dims(D=32))) == 0
+    # q, k, v, sinks, cu_seqlens, window, scale, out, lse, dout, dq, dk, dv, dsinks
+    args = [FAKE] * 4 + [None, 0, ctypes.c_float(0.125)] + [FAKE] * 7
+    # workspace too small
+    assert L.sink_attn_bwd(ctypes.byref(d), *args, FAKE, ctypes.c_size_t(ws - 1), None) == 7
+    assert L.sink_attn_bwd(ctypes.byref(d), *args, None, ctypes.c_size_t(ws), None) == 7
+    # workspace misaligned
+    assert L.sink_attn_bwd(ctypes.byref(d), *args, ctypes.c_void_p((1 << 20) + 16), ctypes.c_size_t(ws), None) == 3
+    # dsinks NULL
+    a2 = list(args)
+    a2[13] = None
+    assert L.sink_attn_bwd(ctypes.byref(d), *a2, FAKE, ctypes.c_size_t(ws), None) == 1
+
+
+def test_launch_counts(L):
+    assert L.sink_attn_fwd_launches(ctypes.byref(dims())) == 1
+    assert L.sink_attn_fwd_launches(ctypes.byref(dims(T=0, batch=0, max_seqlen=0))) == 0
+    assert L.sink_attn_bwd_launches(ctypes.byref(dims())) >= 0
