@@ -50,3 +50,20 @@ def run_fwd(w, arrays, ops, stream=None):
     torch.cuda.synchronize()
     assert ops.device_error() == 0
     return out, lse
+
+
+def run_bwd(w, arrays, ops, out, lse, stream=None):
+    """sink_attn_bwd on the workload's arrays with the forward's saved
+    out / lse; returns (dq, dk, dv, dsinks) tensors."""
+    q, k, v = dev_bf16(arrays["q"]), dev_bf16(arrays["k"]), dev_bf16(arrays["v"])
+    s = dev(arrays["sinks"])
+    do = dev_bf16(arrays["dout"])
+    if w.uniform_seqlen is not None:
+        r = ops.bwd(q, k, v, s, out, lse, do, None, w.window, w.scale, batch=w.batch,
+                    max_seqlen=w.uniform_seqlen, stream=stream)
+    else:
+        cu = dev(w.cu_seqlens)
+        r = ops.bwd(q, k, v, s, out, lse, do, cu, w.window, w.scale, max_seqlen=w.max_seqlen, stream=stream)
+    torch.cuda.synchronize()
+    assert ops.device_error() == 0
+    return r
