@@ -1,0 +1,405 @@
+"""Benchmark of the sink-attention hot path on B200.
+
+One step = forward + backward of one sliding-window layer (window 128) and
+one full-causal layer of gpt-oss attention shapes (B=4, S=4096, 64 query
+heads, 8 key/value heads, head dim 64, scale 1/8), on synthetic seeded bf16
+inputs already resident in HBM.  The metric is TFLOP/s on unmasked FLOPs
+(forward 4*D per allowed (query, key, head) triple, backward 10*D), counted
+exactly from the mask.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+With N > 1 (launched by torchrun) every rank runs its own replica of the
+workload on its own GPU (the path has no exchange step: replicas only, weak
+scaling); the reported time is the max over ranks.  Rank 0 prints one JSON
+line.
+
+--impl reference times the fp64 CPU oracle (the correctness reference) on a
+bounded sample of the same workload on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from sink_sliding_window_b200 import synth  # noqa: E402
+
+WORKLOAD = "prefill4k"
+B, S, HQ, HKV, D = 4, 4096, 64, 8, 64
+LAYERS = (128, 0)  # window per layer: sliding window 128, then full causal
+METRIC = "sink-attn fwd/bwd TFLOP/s (unmasked FLOPs) and % of B200 bf16 tensor peak"
+
+
+# ------------------------------------------------------------------ work
+def pairs(cu_seqlens, window, Hq):
+    """Allowed (query, key, head) triples, counted exactly from the mask."""
+    c = np.asarray(cu_seqlens, np.int64)
+    tot = 0
+    for b in range(len(c) - 1):
+        i = np.arange(int(c[b + 1] - c[b]), dtype=np.int64)
+        n = i + 1 if window <= 0 else np.minimum(i + 1, window)
+        tot += int(n.sum())
+    return tot * Hq
+
+
+def layer_flops(window):
+    p = pairs(synth.uniform_cu_seqlens(B, S), window, HQ)
+    return 4 * D * p, 10 * D * p
+
+
+def step_flops():
+    return sum(sum(layer_flops(w)) for w in LAYERS)
+
+
+# ------------------------------------------------------------- CPU sample
+_SAMPLE_CACHE = {}
+
+
+def _sample_inputs(seed):
+    if seed not in _SAMPLE_CACHE:
+        _SAMPLE_CACHE[seed] = synth.workload(f"{WORKLOAD}:w128", seed=seed).generate(with_dout=True)
+    return _SAMPLE_CACHE[seed]
+
+
+def oracle_sample(len_window=S, len_full=1024, seed=0, nthreads=0):
+    """Bounded sample of the workload for the CPU oracle: forward+backward
+    (the oracle's backward recomputes the forward rows) restricted to 4 of
+    the 8 key/value heads (and their 32 query heads), all 4 documents:
+      - the window-128 layer on the first `len_window` tokens of each
+        document, and
+      - the full-causal layer on the first `len_full` tokens of each document.
+    The oracle parallelises over (document, key/value head) tasks: 16 here.
+    Returns (seconds, flops, description, threads)."""
+    import oracle
+
+    a = _sample_inputs(seed)
+    G = HQ // HKV
+    groups = [0, 2, 5, 7]
+    heads = np.concatenate([np.arange(g * G, (g + 1) * G) for g in groups])
+    flops = 0
+    secs = 0.0
+    for window, length in ((128, len_window), (0, len_full)):
+        rows = np.concatenate([np.arange(b * S, b * S + length) for b in range(B)])
+        q = np.ascontiguousarray(a["q"][rows][:, heads])
+        k = np.ascontiguousarray(a["k"][rows][:, groups])
+        v = np.ascontiguousarray(a["v"][rows][:, groups])
+        do = np.ascontiguousarray(a["dout"][rows][:, heads])
+        cu = synth.uniform_cu_seqlens(B, length)
+        t0 = time.perf_counter()
+        oracle.bwd(q, k, v, a["sinks"][heads], cu, window, 1.0 / 8.0, do, nthreads=nthreads)
+        secs += time.perf_counter() - t0
+        flops += (4 + 10) * D * pairs(cu, window, len(heads))
+    desc = (f"fp64 oracle fwd+bwd, 4 documents x 4 of 8 KV heads (32 query heads): window-128 layer on the first "
+            f"{len_window} tokens and full-causal layer on the first {len_full} tokens of each document")
+    return secs, flops, desc, oracle.max_threads() if nthreads <= 0 else nthreads
+
+
+# ----------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during a region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu_id}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 7:
+                continue
+            try:
+                sm.append(float(f[0]))
+                smax.append(float(f[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[3:7]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def gpu_id_for(torch, dev):
+    try:
+        p = torch.cuda.get_device_properties(dev)
+        return f"{p.pci_domain_id:08X}:{p.pci_bus_id:02X}:{p.pci_device_id:02X}.0"
+    except Exception:
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+        return vis.split(",")[dev] if vis else str(dev)
+
+
+# ---------------------------------------------------------------- helpers
+def read_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            pk = json.load(f)
+        return float(pk["bf16_tflops"]), float(pk["hbm_gbs"]), "measured"
+    return 1590.0, 6650.0, "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "sink_sliding_window_b200", "csrc")
+    for n in sorted(os.listdir(csrc)):
+        if n.endswith((".cu", ".cuh")):
+            with open(os.path.join(csrc, n), "rb") as f:
+                h.update(n.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic():
+    """DRAM bytes per launch of the backward main kernel on this workload,
+    from the committed ncu summary; None when the kernels changed since."""
+    path = os.path.join(ROOT, "profiles", "bwd_main_prefill4k_full.traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        t = json.load(f)
+    return t.get("dram_bytes_per_launch") if t.get("kernel_source_hash") == kernel_source_hash() else None
+
+
+# ------------------------------------------------------------------- arms
+def run_reference(args, rank):
+    if rank != 0:
+        return
+    # Size each step so that all warmup + timed steps take about two minutes:
+    # the sample's work grows ~linearly with the window-layer prefix and
+    # quadratically with the full-causal prefix.
+    budget = 120.0 / (args.warmup + args.steps)
+    secs1, _, _, _ = oracle_sample(256, 256)  # calibration, untimed
+    lw, lf = 256, 256
+    while lw < S and secs1 * (2 * lw / 256 + (lf / 256) ** 2) / 3 * 2 < budget:
+        lw, lf = 2 * lw, min(1024, 2 * lf)
+    steps = []
+    for i in range(args.warmup + args.steps):
+        secs, flops, desc, threads = oracle_sample(lw, lf)
+        if i >= args.warmup:
+            steps.append((secs, flops))
+    secs = sum(s for s, _ in steps)
+    flops = sum(f for _, f in steps)
+    value = flops / secs / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / len(steps),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_dict(),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": desc},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def config_dict():
+    return {"workload": f"{WORKLOAD}: B=4 S=4096 Hq=64 Hkv=8 D=64 scale=1/8, one window-128 layer + one "
+                        f"full-causal layer, forward+backward",
+            "batch": B, "seq_len": S, "num_q_heads": HQ, "num_kv_heads": HKV, "head_dim": D,
+            "windows": list(LAYERS), "parallelism": "replicas (one independent workload per GPU)",
+            "l2": "no flush; per-step working set (q,k,v,dout,out,lse,dq accumulator ~ 1 GB) exceeds the 126 MB L2"}
+
+
+def run_ours(args, rank, world, torch, dist):
+    from sink_sliding_window_b200 import build, ops
+
+    dev = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(dev)
+    build.build()
+    ops.load()
+    w = synth.workload(f"{WORKLOAD}:w128", seed=rank)
+    a = w.generate(with_dout=True)
+
+    def to_dev(bits):
+        return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).cuda()
+
+    q, k, v, dout = to_dev(a["q"]), to_dev(a["k"]), to_dev(a["v"]), to_dev(a["dout"])
+    sinks = torch.from_numpy(a["sinks"]).cuda()
+    T = B * S
+    outs = {W: (torch.empty_like(q), torch.empty((HQ, T), dtype=torch.float32, device="cuda")) for W in LAYERS}
+    grads = {W: (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v),
+                 torch.empty((HQ,), dtype=torch.float32, device="cuda")) for W in LAYERS}
+    ws = torch.empty((ops.bwd_workspace_size(T, HQ, HKV, D, B, S),), dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+    kw = dict(batch=B, max_seqlen=S, stream=stream)
+
+    def step(q, k, v, sinks, dout, prof=None):
+        for W in LAYERS:
+            o, l = outs[W]
+            ops.fwd(q, k, v, sinks, None, W, 0.125, out=o, lse=l, **kw)
+        for W in LAYERS:
+            o, l = outs[W]
+            dq, dk, dv, ds = grads[W]
+            if prof is not None and W == 0:
+                ops.profile_events(ops.PROFILE_BWD_MAIN, *prof)
+            ops.bwd(q, k, v, sinks, o, l, dout, None, W, 0.125, dq=dq, dk=dk, dv=dv, dsinks=ds, workspace=ws, **kw)
+            if prof is not None and W == 0:
+                ops.profile_events(ops.PROFILE_BWD_MAIN)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    # ---- device-resident timing
+    for _ in range(args.warmup):
+        step(q, k, v, sinks, dout)
+    torch.cuda.synchronize()
+    assert ops.device_error() == 0
+    prof = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for b_, e_ in prof:  # torch creates the CUDA event on its first record
+        b_.record(stream)
+        e_.record(stream)
+    clocks = ClockSampler(gpu_id_for(torch, dev))
+    clocks.start()
+    barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(args.steps):
+        step(q, k, v, sinks, dout, prof=prof[i])
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    ms = e0.elapsed_time(e1)
+    kern_ms = float(np.mean([b.elapsed_time(e) for b, e in prof]))
+    if ops.device_error() != 0:
+        raise RuntimeError("a kernel reported a timed-out wait")
+    if dist is not None:
+        t = torch.tensor([ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+
+    flops = step_flops()
+    value = world * flops * args.steps / (ms / 1e3) / 1e12
+    launches = args.steps * len(LAYERS) * (ops.fwd_launches(T, HQ, HKV, D, B, S) + ops.bwd_launches(T, HQ, HKV, D, B, S))
+
+    # ---- end to end through host buffers (pinned), copies inside the region
+    e2e_steps = max(1, min(args.steps, args.e2e_steps))
+    h_in = {n: t.cpu().pin_memory() for n, t in (("q", q), ("k", k), ("v", v), ("dout", dout), ("sinks", sinks))}
+    h_out = [t.cpu().pin_memory() for W in LAYERS for t in (*outs[W], *grads[W])]
+    d_out = [t for W in LAYERS for t in (*outs[W], *grads[W])]
+    h2d = sum(t.numel() * t.element_size() for t in h_in.values())
+    d2h = sum(t.numel() * t.element_size() for t in h_out)
+    barrier()
+    torch.cuda.synchronize()
+    x0, x1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    x0.record(stream)
+    for _ in range(e2e_steps):
+        q.copy_(h_in["q"], non_blocking=True)
+        k.copy_(h_in["k"], non_blocking=True)
+        v.copy_(h_in["v"], non_blocking=True)
+        dout.copy_(h_in["dout"], non_blocking=True)
+        sinks.copy_(h_in["sinks"], non_blocking=True)
+        step(q, k, v, sinks, dout)
+        for h, d in zip(h_out, d_out):
+            h.copy_(d, non_blocking=True)
+    x1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = x0.elapsed_time(x1)
+    if dist is not None:
+        t = torch.tensor([e2e_ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_value = world * flops * e2e_steps / (e2e_ms / 1e3) / 1e12
+
+    if rank != 0:
+        return
+    peak, _, peak_kind = read_peaks()
+    fwd_full, bwd_full = layer_flops(0)
+    achieved = bwd_full / (kern_ms / 1e3) / 1e12
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) bf16 q/k/v/dout, N(0,1) sinks)",
+        "config": config_dict(),
+        "pct_of_peak": 100.0 * value / world / peak,
+        "roofline": {"bound": "tensor", "kernel": "sink_attn_bwd_main (full-causal layer)",
+                     "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                     "peak_source": f"{peak_kind} bf16_tflops (burst)", "traffic": measured_traffic(),
+                     "flops_per_launch": bwd_full, "avg_launch_ms": kern_ms},
+        "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "steps": e2e_steps},
+        "gpu_launches": launches,
+        "clocks": clk,
+    }
+    if world == 1 and not args.skip_cpu_baseline:
+        secs, cflops, desc, threads = oracle_sample()
+        line["cpu_baseline"] = {"value": cflops / secs / 1e12, "unit": "TFLOP/s", "cores": threads,
+                                "kind": "oracle", "sample": desc, "seconds": secs}
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--skip-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank)
+        return 0
+    import torch
+
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist_
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+        dist_.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        dist = dist_
+    try:
+        run_ours(args, rank, world, torch, dist)
+    finally:
+        if dist is not None:
+            dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

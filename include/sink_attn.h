@@ -122,6 +122,14 @@ const char* sink_attn_status_string(sink_attn_status s);
  * entry point that synchronises. */
 int sink_attn_device_error(void* stream);
 
+/* Profiling aid.  Registers two CUDA events (cudaEvent_t passed as void*)
+ * that later calls record on their stream immediately before and after one
+ * kernel launch: which = 0 -> the forward kernel of sink_attn_fwd,
+ * which = 1 -> the main (tensor-core) kernel of sink_attn_bwd.  Passing NULL
+ * events clears the slot.  Process-wide and not thread-safe; the events stay
+ * owned by the caller.  Returns SINK_ATTN_ERR_SHAPE for an unknown `which`. */
+sink_attn_status sink_attn_profile_events(int which, void* ev_begin, void* ev_end);
+
 /* Number of kernels one sink_attn_fwd / sink_attn_bwd call launches for
  * these sizes (0 when T = 0). */
 int sink_attn_fwd_launches(const sink_attn_dims* dims);

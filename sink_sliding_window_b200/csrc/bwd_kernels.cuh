@@ -500,7 +500,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 inline sink_attn_status bwd_launch(const Geometry& geo, float scale, const void* q, const void* k, const void* v,
                                    const float* sinks, const void* out, const float* lse, const void* dout, void* dq,
                                    void* dk, void* dv, float* dsinks, uint8_t* ws_base, const BwdWorkspace& ws,
-                                   cudaStream_t stream) {
+                                   cudaStream_t stream, cudaEvent_t ev_main_begin, cudaEvent_t ev_main_end) {
   float* dq_acc = reinterpret_cast<float*>(ws_base + ws.dq_acc);
   float* Dvec = reinterpret_cast<float*>(ws_base + ws.Dvec);
   float* partials = reinterpret_cast<float*>(ws_base + ws.partials);
@@ -547,8 +547,10 @@ inline sink_attn_status bwd_launch(const Geometry& geo, float scale, const void*
   bp.num_key_tiles = (geo.T + kBlockN - 1) / kBlockN;
   const int64_t grid = static_cast<int64_t>(bp.num_key_tiles) * geo.Hkv;
   if (grid > 0x7fffffff) return SINK_ATTN_ERR_UNSUPPORTED;
+  if (ev_main_begin) cudaEventRecord(ev_main_begin, stream);
   sink_attn_bwd_main_kernel<<<static_cast<unsigned>(grid), kBwdThreads, kBwdSmemBytes, stream>>>(tq, tk, tv, tdo,
                                                                                                   bp);
+  if (ev_main_end) cudaEventRecord(ev_main_end, stream);
   if (cudaPeekAtLastError() != cudaSuccess) return SINK_ATTN_ERR_CUDA;
 
   // 3. finish

@@ -62,6 +62,9 @@ sink_attn_status check_dims(const sink_attn_dims* d, const int* cu_seqlens, bool
   return SINK_ATTN_OK;
 }
 
+// Events registered by sink_attn_profile_events: [which][begin/end].
+cudaEvent_t g_profile_events[2][2] = {{nullptr, nullptr}, {nullptr, nullptr}};
+
 template <typename K>
 bool set_smem_once(K kernel, size_t bytes, int* done_flag) {
   // Per process; the attribute is per function, not per device context.
@@ -92,6 +95,13 @@ const char* sink_attn_status_string(sink_attn_status s) {
     case SINK_ATTN_ERR_WORKSPACE: return "workspace missing or too small";
   }
   return "unknown status";
+}
+
+sink_attn_status sink_attn_profile_events(int which, void* ev_begin, void* ev_end) {
+  if (which < 0 || which > 1) return SINK_ATTN_ERR_SHAPE;
+  g_profile_events[which][0] = static_cast<cudaEvent_t>(ev_begin);
+  g_profile_events[which][1] = static_cast<cudaEvent_t>(ev_end);
+  return SINK_ATTN_OK;
 }
 
 int sink_attn_device_error(void* stream) {
@@ -140,8 +150,10 @@ sink_attn_status sink_attn_fwd(const sink_attn_dims* d, const void* q, const voi
   p.lse = lse;
   const int64_t grid = static_cast<int64_t>(geo.num_qblocks) * geo.Hkv;
   if (grid > 0x7fffffff) return SINK_ATTN_ERR_UNSUPPORTED;
-  sink_attn_fwd_kernel<<<static_cast<unsigned>(grid), kFwdThreads, kFwdSmemBytes,
-                         static_cast<cudaStream_t>(stream)>>>(tq, tk, tv, p);
+  cudaStream_t st_ = static_cast<cudaStream_t>(stream);
+  if (g_profile_events[0][0]) cudaEventRecord(g_profile_events[0][0], st_);
+  sink_attn_fwd_kernel<<<static_cast<unsigned>(grid), kFwdThreads, kFwdSmemBytes, st_>>>(tq, tk, tv, p);
+  if (g_profile_events[0][1]) cudaEventRecord(g_profile_events[0][1], st_);
   return cudaPeekAtLastError() == cudaSuccess ? SINK_ATTN_OK : SINK_ATTN_ERR_CUDA;
 }
 
@@ -181,7 +193,8 @@ sink_attn_status sink_attn_bwd(const sink_attn_dims* d, const void* q, const voi
   if (!workspace || workspace_bytes < ws.total) return SINK_ATTN_ERR_WORKSPACE;
   if (reinterpret_cast<uintptr_t>(workspace) & 255u) return SINK_ATTN_ERR_ALIGN;
   return bwd_launch(geo, scale, q, k, v, sinks, out, lse, dout, dq, dk, dv, dsinks,
-                    static_cast<uint8_t*>(workspace), ws, static_cast<cudaStream_t>(stream));
+                    static_cast<uint8_t*>(workspace), ws, static_cast<cudaStream_t>(stream), g_profile_events[1][0],
+                    g_profile_events[1][1]);
 }
 
 }  // extern "C"

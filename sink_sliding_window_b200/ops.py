@@ -26,7 +26,7 @@ STATUS = {
 }
 
 EXPORTS = ("sink_attn_fwd", "sink_attn_bwd", "sink_attn_bwd_workspace_size", "sink_attn_status_string",
-           "sink_attn_device_error", "sink_attn_fwd_launches", "sink_attn_bwd_launches")
+           "sink_attn_device_error", "sink_attn_fwd_launches", "sink_attn_bwd_launches", "sink_attn_profile_events")
 
 
 class SinkAttnError(RuntimeError):
@@ -69,6 +69,8 @@ def load():
         L.sink_attn_fwd_launches.restype = I
         L.sink_attn_bwd_launches.argtypes = [DP]
         L.sink_attn_bwd_launches.restype = I
+        L.sink_attn_profile_events.argtypes = [I, P, P]
+        L.sink_attn_profile_events.restype = I
         _lib = L
     return _lib
 
@@ -166,3 +168,21 @@ def fwd_launches(T, Hq, Hkv, D, batch, max_seqlen) -> int:
 def bwd_launches(T, Hq, Hkv, D, batch, max_seqlen) -> int:
     d = make_dims(T, Hq, Hkv, D, batch, max_seqlen)
     return int(load().sink_attn_bwd_launches(ctypes.byref(d)))
+
+
+PROFILE_FWD = 0
+PROFILE_BWD_MAIN = 1
+
+
+def profile_events(which: int, begin=None, end=None) -> None:
+    """Registers torch.cuda.Event objects (created with enable_timing=True)
+    that the library records right before and after one kernel launch
+    (PROFILE_FWD: the forward kernel; PROFILE_BWD_MAIN: the backward's
+    tensor-core kernel).  profile_events(which) clears the slot."""
+    if (begin is not None and not begin.cuda_event) or (end is not None and not end.cuda_event):
+        raise ValueError("record each event once before registering it (torch creates it on first record)")
+    b = None if begin is None else ctypes.c_void_p(begin.cuda_event)
+    e = None if end is None else ctypes.c_void_p(end.cuda_event)
+    st = load().sink_attn_profile_events(int(which), b, e)
+    if st != 0:
+        raise SinkAttnError(st, "sink_attn_profile_events")
