@@ -114,6 +114,43 @@ sink_attn_status sink_attn_bwd(const sink_attn_dims* dims,
                                void* workspace, size_t workspace_bytes,
                                void* stream);
 
+/* Size of the library's built-in backward scratch buffer used by
+ * sink_attn_bwd_noalloc(): 32 MiB. */
+#define SINK_ATTN_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+
+/* Backward for callers that cannot allocate device memory.  This entry point
+ * is an addition of this library; the pages describe nothing like it.
+ *
+ * Some callers cannot call cudaMalloc or hand over a workspace: code running
+ * inside a memory pool or allocator callback that must not re-enter the
+ * allocator, host code that is not allowed to grow device memory after
+ * start-up, or a binding whose only way to pass memory is the tensors it
+ * already owns.  This entry point computes exactly what sink_attn_bwd()
+ * computes, with the same arguments minus the workspace: its scratch (fp32 dq
+ * accumulator, D_i, sink partials) lives in a fixed array of
+ * SINK_ATTN_NOALLOC_SCRATCH_BYTES inside the library, which every GPU that
+ * loads the library holds until the process exits.  It calls no cudaMalloc,
+ * cudaFree or other allocating routine.
+ *
+ *  - Sizes whose sink_attn_bwd_workspace_size() exceeds the array are refused
+ *    with SINK_ATTN_ERR_WORKSPACE before any launch (at 64 query heads and
+ *    head dim 64 that is about 2000 tokens; at 8 query heads about 16000).
+ *  - The first call on each device looks up the array's device address
+ *    (cudaGetSymbolAddress, with that device current); make that first call
+ *    before capturing a stream into a CUDA graph.
+ *  - Every call on a device shares the one array and leaves its contents
+ *    behind; the kernels re-initialise everything they read (the dq
+ *    accumulator is zeroed each call).  Calls whose execution overlaps on the
+ *    GPU (different streams, or different host threads) race on the array and
+ *    give wrong results: serialise them. */
+sink_attn_status sink_attn_bwd_noalloc(const sink_attn_dims* dims,
+                                       const void* q, const void* k, const void* v,
+                                       const float* sinks, const int* cu_seqlens,
+                                       int window, float scale,
+                                       const void* out, const float* lse, const void* dout,
+                                       void* dq, void* dk, void* dv, float* dsinks,
+                                       void* stream);
+
 /* Human-readable name of a status code (static string, never NULL). */
 const char* sink_attn_status_string(sink_attn_status s);
 

@@ -198,3 +198,48 @@ sink_attn_status sink_attn_bwd(const sink_attn_dims* d, const void* q, const voi
 }
 
 }  // extern "C"
+
+// ----------------------------------------------------------------------------
+// Backward without caller-provided workspace, for callers that cannot
+// allocate device memory (see sink_attn_bwd_noalloc in sink_attn.h).  The
+// scratch is this fixed array; host code must not use its name as a device
+// address (it is a host-side stand-in), so its address is looked up once per
+// device with cudaGetSymbolAddress and cached.
+namespace {
+
+static __device__ __align__(256) uint8_t g_noalloc_scratch[SINK_ATTN_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mutex;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of g_noalloc_scratch on the current device, or nullptr.
+void* noalloc_scratch_for_current_device() {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || ptr == nullptr) return nullptr;
+    g_noalloc_ptr[dev] = ptr;
+  }
+  return g_noalloc_ptr[dev];
+}
+
+}  // namespace
+
+extern "C" sink_attn_status sink_attn_bwd_noalloc(const sink_attn_dims* d, const void* q, const void* k,
+                                                  const void* v, const float* sinks, const int* cu_seqlens,
+                                                  int window, float scale, const void* out, const float* lse,
+                                                  const void* dout, void* dq, void* dk, void* dv, float* dsinks,
+                                                  void* stream) {
+  Geometry geo;
+  sink_attn_status st = check_dims(d, cu_seqlens, cu_seqlens != nullptr, window, scale, &geo);
+  if (st != SINK_ATTN_OK) return st;
+  const size_t need = bwd_workspace_layout(geo).total;
+  if (need > SINK_ATTN_NOALLOC_SCRATCH_BYTES) return SINK_ATTN_ERR_WORKSPACE;
+  void* scratch = noalloc_scratch_for_current_device();
+  if (scratch == nullptr) return SINK_ATTN_ERR_CUDA;
+  return sink_attn_bwd(d, q, k, v, sinks, cu_seqlens, window, scale, out, lse, dout, dq, dk, dv, dsinks, scratch,
+                       SINK_ATTN_NOALLOC_SCRATCH_BYTES, stream);
+}
