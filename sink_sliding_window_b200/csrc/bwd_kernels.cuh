@@ -6,16 +6,21 @@
 //   dv_j = sum_{i,h in group} P_ij dout_i,  dsinks_h = -sum_i P_sink,i D_i
 //
 // Three launches on the caller's stream:
-//   1. bwd_preprocess: D_i (fp32, [Hq][T]), per-block partial sums of
-//      -P_sink,i D_i (fixed order), and zeroes the fp32 dq accumulator.
-//   2. bwd_main (tcgen05): one CTA per 128-key tile of one key/value head g.
-//      It visits every query tile (the fwd's 128 rows = 128/G tokens x G
-//      heads) that can see one of its keys and computes, with keys on the
-//      TMEM lanes:  S^T = K Q^T, dP^T = V dO^T (MMA), P and dS (1 thread =
-//      1 key), dV += P^T dO, dK += dS^T Q (MMA, A operand from TMEM: dK and
-//      dV sum over all G heads of the group inside TMEM, no atomics), and
-//      dQ = dS K (MMA, A operand = dS staged in shared memory) which is added
-//      to the fp32 accumulator with vector atomics.
+//   1. bwd_preprocess: D_i; lse_i*log2(e) and D_i re-laid out in query-tile
+//      row order (so the main kernel fetches a tile's 128 values with one bulk
+//      copy); the first allowed key of every token; per-block partial sums of
+//      -P_sink,i D_i (fixed order); and zeroes the fp32 dq accumulator.
+//   2. bwd_main (tcgen05): one CTA per 128-key tile of one key/value head g,
+//      visiting every query tile (the forward's 128 rows = 128/G tokens x G
+//      heads) that can see one of its keys.  Keys sit on the TMEM lanes:
+//        S^T = K Q^T, dP^T = V dO^T          (MMA, fp32 in TMEM)
+//        P = 2^(S^T*scale*log2e - lse2), dS = P (dP - D)   (8 warps)
+//        dV += P^T dO, dK += dS^T Q          (MMA, A from TMEM; dV and dK sum
+//                                             over the G heads inside TMEM)
+//        dQ = dS K                           (MMA, A = dS in shared memory)
+//      dQ tiles are reduced into the fp32 accumulator by TMA reduce-add.
+//      Two S^T buffers let the tensor core compute tile i+2's S^T and tile
+//      i+1's dP^T while the softmax warps work on tile i+1.
 //   3. bwd_finish: dq = bf16(scale * accumulator), and dsinks_h = fixed-order
 //      tree sum of the partials (bitwise reproducible).
 #pragma once
@@ -26,19 +31,15 @@ namespace sa {
 
 constexpr int kBwdLaunches = 3;
 constexpr int kPreThreads = 256;  // tokens per preprocess CTA (one head per CTA)
-constexpr int kBwdThreads = 320;  // 10 warps
-constexpr int kBwdStages = 2;
-constexpr uint32_t kBwdTmemCols = 512;
-constexpr uint32_t kBwdTmemS = 0;     // S^T fp32 [128 keys][128 rows]; P^T (bf16) aliases cols 0..63
-constexpr uint32_t kBwdTmemDP = 128;  // dP^T fp32; dS^T (bf16) aliases cols 128..191
-constexpr uint32_t kBwdTmemDV = 256;  // dV accumulator fp32 [128 keys][64]
-constexpr uint32_t kBwdTmemDK = 320;  // dK accumulator
-constexpr uint32_t kBwdTmemDQ = 384;  // dQ tile fp32 [128 rows][64]
 constexpr int kFinishThreads = 256;
 
+// ---------------------------------------------------------------- workspace
 struct BwdWorkspace {
   size_t dq_acc;    // fp32 [T][Hq][D]
   size_t Dvec;      // fp32 [Hq][T]
+  size_t lse2_blk;  // fp32 [num_qblocks][Hkv][128]  lse*log2(e) in tile-row order (+inf for padding rows)
+  size_t D_blk;     // fp32 [num_qblocks][Hkv][128]  D in tile-row order (0 for padding rows)
+  size_t lo_blk;    // int  [num_qblocks][128]       first allowed key per token of the tile
   size_t partials;  // fp32 [Hq][num_pre_blocks]
   int num_pre_blocks;
   size_t total;
@@ -49,24 +50,36 @@ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 inline BwdWorkspace bwd_workspace_layout(const Geometry& geo) {
   BwdWorkspace w;
   const size_t T = static_cast<size_t>(geo.T);
-  w.num_pre_blocks = static_cast<int>((T + kPreThreads - 1) / kPreThreads);
-  w.dq_acc = 0;
-  w.Dvec = align_up(T * geo.Hq * kHeadDim * sizeof(float), 256);
-  w.partials = w.Dvec + align_up(T * geo.Hq * sizeof(float), 256);
-  w.total = w.partials + align_up(static_cast<size_t>(geo.Hq) * (w.num_pre_blocks > 0 ? w.num_pre_blocks : 1) *
-                                      sizeof(float),
-                                  256);
+  const size_t T_pad = static_cast<size_t>(geo.num_qblocks) << geo.P_log2;
+  w.num_pre_blocks = static_cast<int>((T_pad + kPreThreads - 1) / kPreThreads);
+  size_t off = 0;
+  w.dq_acc = off;
+  off += align_up(T * geo.Hq * kHeadDim * sizeof(float), 256);
+  w.Dvec = off;
+  off += align_up(T * geo.Hq * sizeof(float), 256);
+  w.lse2_blk = off;
+  off += align_up(static_cast<size_t>(geo.num_qblocks) * geo.Hkv * kBlockM * sizeof(float), 256);
+  w.D_blk = off;
+  off += align_up(static_cast<size_t>(geo.num_qblocks) * geo.Hkv * kBlockM * sizeof(float), 256);
+  w.lo_blk = off;
+  off += align_up(static_cast<size_t>(geo.num_qblocks) * kBlockM * sizeof(int), 256);
+  w.partials = off;
+  off += align_up(static_cast<size_t>(geo.Hq) * (w.num_pre_blocks > 0 ? w.num_pre_blocks : 1) * sizeof(float), 256);
+  w.total = off;
   return w;
 }
 
 // ------------------------------------------------------------ preprocess
 struct PreParams {
-  int T, Hq;
+  Geometry geo;
   const __nv_bfloat16* out;
   const __nv_bfloat16* dout;
   const float* lse;
   const float* sinks;
   float* Dvec;
+  float* lse2_blk;
+  float* D_blk;
+  int* lo_blk;
   float* partials;
   float* dq_acc;
   int num_pre_blocks;
@@ -86,26 +99,44 @@ __device__ __forceinline__ float dot8_bf16(uint4 a, uint4 b) {
   return s;
 }
 
-// Grid (num_pre_blocks, Hq); thread = one token of head blockIdx.y.
+// Grid (num_pre_blocks, Hq); thread = one token (padded up to whole query
+// tiles) of head blockIdx.y.
 __global__ void __launch_bounds__(kPreThreads) sink_attn_bwd_preprocess_kernel(const PreParams p) {
   __shared__ float warp_sums[kPreThreads / 32];
+  const Geometry& geo = p.geo;
   const int h = blockIdx.y;
   const int t = blockIdx.x * kPreThreads + threadIdx.x;
+  const int t_pad = geo.num_qblocks << geo.P_log2;
   float contrib = 0.f;
-  if (t < p.T) {
-    const size_t row = (static_cast<size_t>(t) * p.Hq + h) * kHeadDim;
-    const uint4* o = reinterpret_cast<const uint4*>(p.out + row);
-    const uint4* g = reinterpret_cast<const uint4*>(p.dout + row);
-    float D = 0.f;
+  if (t < t_pad) {
+    const int qb = t >> geo.P_log2;
+    const int pos = t & ((1 << geo.P_log2) - 1);
+    const int g = h >> geo.G_log2;
+    const int r = (pos << geo.G_log2) + (h & ((1 << geo.G_log2) - 1));
+    const size_t bi = (static_cast<size_t>(qb) * geo.Hkv + g) * kBlockM + r;
+    if (t < geo.T) {
+      const size_t row = (static_cast<size_t>(t) * geo.Hq + h) * kHeadDim;
+      const uint4* o = reinterpret_cast<const uint4*>(p.out + row);
+      const uint4* gr = reinterpret_cast<const uint4*>(p.dout + row);
+      float D = 0.f;
 #pragma unroll
-    for (int i = 0; i < kHeadDim / 8; ++i) D += dot8_bf16(__ldg(o + i), __ldg(g + i));
-    p.Dvec[static_cast<size_t>(h) * p.T + t] = D;
-    const float lse = __ldg(p.lse + static_cast<size_t>(h) * p.T + t);
-    const float psink = ex2_approx((__ldg(p.sinks + h) - lse) * kLog2e);  // e^{s_h - lse}; 0 for s = -inf
-    contrib = -psink * D;
-    float4* acc = reinterpret_cast<float4*>(p.dq_acc + row);
+      for (int i = 0; i < kHeadDim / 8; ++i) D += dot8_bf16(__ldg(o + i), __ldg(gr + i));
+      const float lse = __ldg(p.lse + static_cast<size_t>(h) * geo.T + t);
+      p.Dvec[static_cast<size_t>(h) * geo.T + t] = D;
+      p.D_blk[bi] = D;
+      p.lse2_blk[bi] = lse * kLog2e;
+      const float psink = ex2_approx((__ldg(p.sinks + h) - lse) * kLog2e);  // e^{s_h - lse}; 0 for s = -inf
+      contrib = -psink * D;
+      float4* acc = reinterpret_cast<float4*>(p.dq_acc + row);
 #pragma unroll
-    for (int i = 0; i < kHeadDim / 4; ++i) acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int i = 0; i < kHeadDim / 4; ++i) acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (h == 0) p.lo_blk[static_cast<size_t>(qb) * kBlockM + pos] = first_key(geo, t);
+    } else {
+      // padding rows of the last query tile: P = 0 and dS = 0 there
+      p.D_blk[bi] = 0.f;
+      p.lse2_blk[bi] = INFINITY;
+      if (h == 0) p.lo_blk[static_cast<size_t>(qb) * kBlockM + pos] = 0x7fffffff;
+    }
   }
   // Fixed-order block reduction: butterfly within each warp, then warps in
   // index order.
@@ -166,41 +197,63 @@ __global__ void __launch_bounds__(kFinishThreads) sink_attn_bwd_finish_kernel(co
 }
 
 // ------------------------------------------------------------------ main
+constexpr int kBwdThreads = 448;    // 14 warps
+constexpr int kBwdStages = 3;       // Q/dO/aux ring
+constexpr int kBwdWarpProducer = 8;
+constexpr int kBwdWarpMma = 9;
+constexpr int kBwdWarpDq0 = 10;     // warps 10..13
+constexpr uint32_t kBwdTmemCols = 512;
+constexpr uint32_t kBwdTmemS0 = 0;    // S^T buffer 0: fp32 [128 keys][128 rows]; P^T bf16 in cols 0..63,
+constexpr uint32_t kBwdTmemS1 = 128;  //   the tile's dQ (fp32 [128 rows][64]) later in cols 64..127
+constexpr uint32_t kBwdTmemDP = 256;  // dP^T fp32; dS^T bf16 in cols 0..31 (rows 0-63) and 64..95 (rows 64-127)
+constexpr uint32_t kBwdTmemDV = 384;  // dV accumulator fp32 [128 keys][64]
+constexpr uint32_t kBwdTmemDK = 448;  // dK accumulator
+
 struct BwdParams {
   Geometry geo;
   float scale;
   float scale_log2;
-  const float* lse;    // [Hq][T]
-  const float* Dvec;   // [Hq][T]
-  float* dq_acc;       // [T][Hq][D] fp32
+  const float* lse2_blk;
+  const float* D_blk;
+  const int* lo_blk;
   __nv_bfloat16* dk;   // [T][Hkv][D]
   __nv_bfloat16* dv;
-  int num_key_tiles;
 };
 
 struct BwdAux {
-  float lse2[kBlockM];  // lse * log2(e) per row (+inf for padding rows)
+  float lse2[kBlockM];  // lse*log2(e) per row of the query tile
   float D[kBlockM];
-  int lo[kBlockM];      // first allowed key per position of the tile
+  int lo[kBlockM];      // first allowed key per token of the tile (first 128/G entries)
 };
 
 struct BwdCtl {
   uint64_t kv_full;
   uint64_t qdo_full[kBwdStages];
   uint64_t qdo_empty[kBwdStages];
-  uint64_t aux_full[kBwdStages];
-  uint64_t s_full;
+  uint64_t s_full[2];
+  uint64_t dp_full;
   uint64_t p_full;
   uint64_t dq_full;
   uint64_t dq_empty;
   uint64_t kd_full;
+  uint64_t pair_sync[4];  // the two softmax warps of one TMEM lane group (64 threads)
+  uint64_t dq_sync;       // the four dQ warps (128 threads)
   uint32_t tmem_base;
   int abort;
 };
 
-// K, V, Q x2, dO x2, dS (two 16 KB halves) + aux + control.
+// Barrier over the threads counted by `bar` (each arrives once per use),
+// with the same bounded wait as every other wait in these kernels.
+__device__ __forceinline__ bool group_sync(uint64_t* bar, uint32_t& phase, volatile int* abort, int code) {
+  mbar_arrive(bar);
+  const bool ok = mbar_wait(bar, phase, abort, &g_device_error, code);
+  phase ^= 1u;
+  return ok;
+}
+
+// K, V, Q x3, dO x3, dS (32 KB), dQ staging (32 KB), aux x3, control.
 constexpr size_t kBwdSmemBytes =
-    1024 + kTileBytes * (2 + 2 * kBwdStages + 2) + sizeof(BwdAux) * kBwdStages + sizeof(BwdCtl);
+    1024 + kTileBytes * (2 + 2 * kBwdStages + 2 + 2) + sizeof(BwdAux) * kBwdStages + sizeof(BwdCtl);
 
 __device__ __forceinline__ int doc_end(const Geometry& g, int t) {
   if (g.cu_seqlens == nullptr) return (t / g.seqlen + 1) * g.seqlen;
@@ -213,20 +266,26 @@ __device__ __forceinline__ int doc_end(const Geometry& g, int t) {
 }
 
 struct BwdTile {
-  int g, k0, k_last, qb0, nq;
+  int g, k0, qb0, nq;
 };
 
-__device__ __forceinline__ BwdTile bwd_tile(const Geometry& geo, int num_key_tiles) {
+__device__ __forceinline__ BwdTile bwd_tile(const Geometry& geo) {
   BwdTile w;
   w.g = blockIdx.x % geo.Hkv;
-  const int n = blockIdx.x / geo.Hkv;  // earlier keys are seen by more queries: they go first
+  int n = blockIdx.x / geo.Hkv;
+  // Key tiles early in their document are seen by the most query tiles: with
+  // equal-length documents hand out the first tile of every document, then
+  // the second, ... (longest first).
+  if (geo.cu_seqlens == nullptr && (geo.seqlen % kBlockN) == 0) {
+    const int per_doc = geo.seqlen / kBlockN;
+    n = (n % geo.batch) * per_doc + n / geo.batch;
+  }
   w.k0 = n * kBlockN;
-  w.k_last = min(w.k0 + kBlockN - 1, geo.T - 1);
-  int q_hi = doc_end(geo, w.k_last) - 1;
-  if (geo.window > 0) q_hi = min(q_hi, w.k_last + geo.window - 1);
+  const int k_last = min(w.k0 + kBlockN - 1, geo.T - 1);
+  int q_hi = doc_end(geo, k_last) - 1;
+  if (geo.window > 0) q_hi = min(q_hi, k_last + geo.window - 1);
   w.qb0 = w.k0 >> geo.P_log2;
   w.nq = (q_hi >> geo.P_log2) - w.qb0 + 1;
-  (void)num_key_tiles;
   return w;
 }
 
@@ -242,7 +301,7 @@ __device__ __forceinline__ uint32_t ds_smem_offset(int key, int chunk16) {
 __global__ void __launch_bounds__(kBwdThreads, 1)
     sink_attn_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                              const BwdParams p) {
+                              const __grid_constant__ CUtensorMap tm_dq, const BwdParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   uint8_t* sK = smem;
@@ -250,30 +309,33 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   uint8_t* sQ = sV + kTileBytes;                  // [kBwdStages]
   uint8_t* sDO = sQ + kBwdStages * kTileBytes;    // [kBwdStages]
   uint8_t* sDS = sDO + kBwdStages * kTileBytes;   // 32 KB
-  BwdAux* aux = reinterpret_cast<BwdAux*>(sDS + 2 * kTileBytes);
+  uint8_t* sDQ = sDS + 2 * kTileBytes;            // 32 KB: two {32 fp32 x 128 rows} swizzled halves
+  BwdAux* aux = reinterpret_cast<BwdAux*>(sDQ + 2 * kTileBytes);
   BwdCtl* ctl = reinterpret_cast<BwdCtl*>(aux + kBwdStages);
   volatile int* abort = &ctl->abort;
   const int warp = threadIdx.x >> 5;
   const Geometry& geo = p.geo;
-  const BwdTile w = bwd_tile(geo, p.num_key_tiles);
-  const int G = 1 << geo.G_log2;
+  const BwdTile w = bwd_tile(geo);
 
   if (threadIdx.x == 0) {
     mbar_init(&ctl->kv_full, 1);
     for (int s = 0; s < kBwdStages; ++s) {
       mbar_init(&ctl->qdo_full[s], 1);
       mbar_init(&ctl->qdo_empty[s], 1);
-      mbar_init(&ctl->aux_full[s], 128);
     }
-    mbar_init(&ctl->s_full, 1);
-    mbar_init(&ctl->p_full, 128);
+    mbar_init(&ctl->s_full[0], 1);
+    mbar_init(&ctl->s_full[1], 1);
+    mbar_init(&ctl->dp_full, 1);
+    mbar_init(&ctl->p_full, 256);
     mbar_init(&ctl->dq_full, 1);
     mbar_init(&ctl->dq_empty, 128);
     mbar_init(&ctl->kd_full, 1);
+    for (int l = 0; l < 4; ++l) mbar_init(&ctl->pair_sync[l], 64);
+    mbar_init(&ctl->dq_sync, 128);
     ctl->abort = 0;
     fence_mbar_init();
   }
-  if (warp == 5) {
+  if (warp == kBwdWarpMma) {
     tmem_alloc(&ctl->tmem_base, kBwdTmemCols);
     tmem_relinquish();
   }
@@ -282,7 +344,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   tc_fence_after();
   const uint32_t tmem = ctl->tmem_base;
 
-  if (warp == 4) {
+  if (warp == kBwdWarpProducer) {
     // ---------------------------------------------------------- TMA producer
     if (elect_one()) {
       tma_prefetch_desc(&tm_q);
@@ -296,175 +358,235 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             !mbar_wait(&ctl->qdo_empty[s], ((i / kBwdStages) - 1) & 1, abort, &g_device_error,
                        kDevErrTimeoutProducer))
           break;
-        const int q0 = (w.qb0 + i) << geo.P_log2;
-        mbar_arrive_expect_tx(&ctl->qdo_full[s], 2 * kTileBytes);
+        const int qb = w.qb0 + i;
+        const int q0 = qb << geo.P_log2;
+        const size_t blk = (static_cast<size_t>(qb) * geo.Hkv + w.g) * kBlockM;
+        mbar_arrive_expect_tx(&ctl->qdo_full[s], 2 * kTileBytes + 3 * kBlockM * 4);
         tma_load_3d(sQ + s * kTileBytes, &tm_q, &ctl->qdo_full[s], 0, w.g << geo.G_log2, q0);
         tma_load_3d(sDO + s * kTileBytes, &tm_do, &ctl->qdo_full[s], 0, w.g << geo.G_log2, q0);
+        bulk_load(aux[s].lse2, p.lse2_blk + blk, kBlockM * 4, &ctl->qdo_full[s]);
+        bulk_load(aux[s].D, p.D_blk + blk, kBlockM * 4, &ctl->qdo_full[s]);
+        bulk_load(aux[s].lo, p.lo_blk + static_cast<size_t>(qb) * kBlockM, kBlockM * 4, &ctl->qdo_full[s]);
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == kBwdWarpMma) {
     // ------------------------------------------------------------ MMA issuer
     if (elect_one()) {
       constexpr uint32_t idesc_s = make_idesc_bf16(kBlockN, kBlockM, 0, 0);    // M=128 keys, N=128 rows
       constexpr uint32_t idesc_acc = make_idesc_bf16(kBlockN, kHeadDim, 0, 1); // A tmem (K-major), B MN-major
       constexpr uint32_t idesc_dq = make_idesc_bf16(kBlockM, kHeadDim, 1, 1);  // A smem MN-major, B MN-major
-      const uint32_t tS = tmem + kBwdTmemS, tDP = tmem + kBwdTmemDP;
-      const uint32_t tDV = tmem + kBwdTmemDV, tDK = tmem + kBwdTmemDK, tDQ = tmem + kBwdTmemDQ;
+      const uint32_t tS0 = tmem + kBwdTmemS0, tS1 = tmem + kBwdTmemS1;
+      const uint32_t tDP = tmem + kBwdTmemDP, tDV = tmem + kBwdTmemDV, tDK = tmem + kBwdTmemDK;
       const uint32_t k_addr = smem_u32(sK), v_addr = smem_u32(sV), ds_addr = smem_u32(sDS);
-      bool ok = mbar_wait(&ctl->kv_full, 0, abort, &g_device_error, kDevErrTimeoutMma);
-      for (int i = 0; ok && i < w.nq; ++i) {
-        const int s = i % kBwdStages;
-        ok = mbar_wait(&ctl->qdo_full[s], (i / kBwdStages) & 1, abort, &g_device_error, kDevErrTimeoutMma);
-        if (!ok) break;
-        tc_fence_after();
-        const uint32_t q_addr = smem_u32(sQ + s * kTileBytes), do_addr = smem_u32(sDO + s * kTileBytes);
-        // S^T = K Q^T and dP^T = V dO^T (both operands K-major over the head dim)
+      auto issue_s = [&](int i) {  // S^T_i = K Q_i^T into buffer i%2
+        const uint32_t q_addr = smem_u32(sQ + (i % kBwdStages) * kTileBytes);
+        const uint32_t d = (i & 1) ? tS1 : tS0;
 #pragma unroll
         for (int kk = 0; kk < kHeadDim / 16; ++kk)
-          mma_ss(tS, make_sdesc_sw128(k_addr + kk * 32, 16, 1024), make_sdesc_sw128(q_addr + kk * 32, 16, 1024),
+          mma_ss(d, make_sdesc_sw128(k_addr + kk * 32, 16, 1024), make_sdesc_sw128(q_addr + kk * 32, 16, 1024),
                  idesc_s, kk > 0);
+      };
+      auto issue_dp = [&](int i) {  // dP^T_i = V dO_i^T
+        const uint32_t do_addr = smem_u32(sDO + (i % kBwdStages) * kTileBytes);
 #pragma unroll
         for (int kk = 0; kk < kHeadDim / 16; ++kk)
-          mma_ss(tDP, make_sdesc_sw128(v_addr + kk * 32, 16, 1024),
-                 make_sdesc_sw128(do_addr + kk * 32, 16, 1024), idesc_s, kk > 0);
-        tc_commit(&ctl->s_full);
+          mma_ss(tDP, make_sdesc_sw128(v_addr + kk * 32, 16, 1024), make_sdesc_sw128(do_addr + kk * 32, 16, 1024),
+                 idesc_s, kk > 0);
+      };
+      auto wait_q = [&](int i) {
+        return mbar_wait(&ctl->qdo_full[i % kBwdStages], (i / kBwdStages) & 1, abort, &g_device_error,
+                         kDevErrTimeoutMma);
+      };
+      bool ok = mbar_wait(&ctl->kv_full, 0, abort, &g_device_error, kDevErrTimeoutMma);
+      if (ok && w.nq > 0) {
+        ok = wait_q(0);
+        if (ok) {
+          tc_fence_after();
+          issue_s(0);
+          tc_commit(&ctl->s_full[0]);
+          issue_dp(0);
+          tc_commit(&ctl->dp_full);
+        }
+      }
+      if (ok && w.nq > 1) {
+        ok = wait_q(1);
+        if (ok) {
+          tc_fence_after();
+          issue_s(1);
+          tc_commit(&ctl->s_full[1]);
+        }
+      }
+      for (int i = 0; ok && i < w.nq; ++i) {
+        const uint32_t tSb = (i & 1) ? tS1 : tS0;
+        const int st = i % kBwdStages;
         ok = mbar_wait(&ctl->p_full, i & 1, abort, &g_device_error, kDevErrTimeoutMma);
         if (!ok) break;
         tc_fence_after();
-        // dV += P^T dO, dK += dS^T Q   (K = the tile's 128 query rows)
+        const uint32_t q_addr = smem_u32(sQ + st * kTileBytes), do_addr = smem_u32(sDO + st * kTileBytes);
+        // dV += P^T dO and dK += dS^T Q over the tile's 128 query rows.  P^T
+        // sits in cols 0..63 of the S^T buffer; dS^T in cols 0..31 (rows
+        // 0-63) and 64..95 (rows 64-127) of the dP^T region.
 #pragma unroll
         for (int kk = 0; kk < kBlockM / 16; ++kk) {
-          mma_ts(tDV, tS + kk * 8, make_sdesc_sw128(do_addr + kk * 2048, kTileBytes, 1024), idesc_acc,
-                 (i > 0 || kk > 0) ? 1u : 0u);
-          mma_ts(tDK, tDP + kk * 8, make_sdesc_sw128(q_addr + kk * 2048, kTileBytes, 1024), idesc_acc,
-                 (i > 0 || kk > 0) ? 1u : 0u);
+          const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
+          mma_ts(tDV, tSb + kk * 8, make_sdesc_sw128(do_addr + kk * 2048, kTileBytes, 1024), idesc_acc, acc);
+          mma_ts(tDK, tDP + (kk < 4 ? kk * 8 : 64 + (kk - 4) * 8),
+                 make_sdesc_sw128(q_addr + kk * 2048, kTileBytes, 1024), idesc_acc, acc);
         }
-        // dQ = dS K   (M = 128 rows, K = 128 keys)
-        if (i > 0) {
-          ok = mbar_wait(&ctl->dq_empty, (i - 1) & 1, abort, &g_device_error, kDevErrTimeoutMma);
-          if (!ok) break;
-          tc_fence_after();
-        }
+        // dQ_i = dS K into the upper half of this tile's S^T buffer
 #pragma unroll
         for (int kk = 0; kk < kBlockN / 16; ++kk)
-          mma_ss(tDQ, make_sdesc_sw128(ds_addr + kk * 2048, 16384, 1024),
+          mma_ss(tSb + 64, make_sdesc_sw128(ds_addr + kk * 2048, 16384, 1024),
                  make_sdesc_sw128(k_addr + kk * 2048, kTileBytes, 1024), idesc_dq, kk > 0);
-        tc_commit(&ctl->qdo_empty[s]);
         tc_commit(&ctl->dq_full);
+        tc_commit(&ctl->qdo_empty[st]);
+        if (i + 1 < w.nq) {
+          // dP^T_{i+1} (dS_i in the dP region was consumed by dK above)
+          ok = wait_q(i + 1);
+          if (!ok) break;
+          tc_fence_after();
+          issue_dp(i + 1);
+          tc_commit(&ctl->dp_full);
+        }
+        if (i + 2 < w.nq) {
+          // S^T_{i+2} reuses this buffer once dQ_i has been read out of it
+          ok = mbar_wait(&ctl->dq_empty, i & 1, abort, &g_device_error, kDevErrTimeoutMma) && wait_q(i + 2);
+          if (!ok) break;
+          tc_fence_after();
+          issue_s(i + 2);
+          tc_commit(&ctl->s_full[i & 1]);
+        }
       }
       if (ok) tc_commit(&ctl->kd_full);
     }
-  } else if (warp < 4) {
-    // ------------------------------------- P / dS (1 thread = 1 key = 1 lane)
-    const int j = w.k0 + threadIdx.x;  // this thread's key
-    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-    const uint32_t tS = tmem + lane_base + kBwdTmemS;
-    const uint32_t tDP = tmem + lane_base + kBwdTmemDP;
+  } else if (warp < 8) {
+    // -------------------- P / dS: 2 warps per TMEM lane group (one key per lane)
+    const int lg = warp & 3;                 // TMEM lane group: keys 32*lg .. 32*lg+31
+    const int ch = warp >> 2;                // query rows [64*ch, 64*ch+64)
+    const int kl = 32 * lg + (threadIdx.x & 31);
+    const int j = w.k0 + kl;                 // this thread's key
+    const uint32_t lane_base = static_cast<uint32_t>(32 * lg) << 16;
     const float sl2 = p.scale_log2;
+    uint32_t pair_phase = 0;
     bool ok = true;
     for (int i = 0; i < w.nq; ++i) {
-      const int s = i % kBwdStages;
-      ok = mbar_wait(&ctl->aux_full[s], (i / kBwdStages) & 1, abort, &g_device_error, kDevErrTimeoutBwd) &&
-           mbar_wait(&ctl->s_full, i & 1, abort, &g_device_error, kDevErrTimeoutBwd);
+      const int st = i % kBwdStages;
+      const uint32_t sbuf = (i & 1) ? kBwdTmemS1 : kBwdTmemS0;
+      ok = mbar_wait(&ctl->qdo_full[st], (i / kBwdStages) & 1, abort, &g_device_error, kDevErrTimeoutSoftmax) &&
+           mbar_wait(&ctl->s_full[i & 1], (i >> 1) & 1, abort, &g_device_error, kDevErrTimeoutSoftmax);
       if (!ok) break;
       tc_fence_after();
-      const BwdAux& a = aux[s];
+      const BwdAux& a = aux[st];
       const int q0 = (w.qb0 + i) << geo.P_log2;
       const int q_last = q0 + (1 << geo.P_log2) - 1;
-      // CTA-uniform: is every (key, row) pair of this block allowed?
+      // CTA-uniform: is every (key, row) pair of this tile allowed?
       const bool full = (w.k0 + kBlockN - 1 < geo.T) && (q_last < geo.T) && (w.k0 + kBlockN - 1 <= q0) &&
-                        (w.k0 >= a.lo[kBlockM / G - 1]);
-#pragma unroll 1
-      for (int c0 = 0; c0 < kBlockM; c0 += 32) {
-        uint32_t sr[32], dr[32];
+                        (w.k0 >= a.lo[(kBlockM >> geo.G_log2) - 1]);
+      const uint32_t tS = tmem + lane_base + sbuf + 64 * ch;
+      const uint32_t tDP = tmem + lane_base + kBwdTmemDP + 64 * ch;
+      float pv[64];
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        uint32_t sr[32];
         __syncwarp();
-        tmem_ld32(tS + c0, sr);
-        tmem_ld32(tDP + c0, dr);
-        uint32_t pk[16], dk[16];
+        tmem_ld32(tS + 32 * half, sr);
 #pragma unroll
-        for (int c = 0; c < 32; c += 2) {
-          float pv[2], dsv[2];
+        for (int c = 0; c < 32; c += 4) {
+          const int col = 64 * ch + 32 * half + c;
+          const float4 l4 = *reinterpret_cast<const float4*>(&a.lse2[col]);
+          const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
 #pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int col = c0 + c + u;
-            float pe = ex2_approx(fmaf(__uint_as_float(sr[c + u]), sl2, -a.lse2[col]));
+          for (int u = 0; u < 4; ++u) {
+            float pe = ex2_approx(fmaf(__uint_as_float(sr[c + u]), sl2, -lv[u]));
             if (!full) {
-              const int pos = col >> geo.G_log2;
-              const int tq = q0 + pos;
-              if (!(j >= a.lo[pos] && j <= tq)) pe = 0.f;
+              const int pos = (col + u) >> geo.G_log2;
+              if (!(j >= a.lo[pos] && j <= q0 + pos)) pe = 0.f;
             }
-            pv[u] = pe;
-            dsv[u] = pe * (__uint_as_float(dr[c + u]) - a.D[col]);
+            pv[32 * half + c + u] = pe;
           }
-          pk[c >> 1] = pack_bf16x2(pv[0], pv[1]);
-          dk[c >> 1] = pack_bf16x2(dsv[0], dsv[1]);
         }
+      }
+      // Both warps of this lane group have read S^T: P^T (bf16) may now
+      // overwrite its first 64 columns.
+      tc_fence_before();
+      ok = group_sync(&ctl->pair_sync[lg], pair_phase, abort, kDevErrTimeoutSoftmax);
+      if (!ok) break;
+      tc_fence_after();
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int c = 0; c < 16; ++c) pk[c] = pack_bf16x2(pv[32 * half + 2 * c], pv[32 * half + 2 * c + 1]);
         __syncwarp();
-        tmem_st16(tS + (c0 >> 1), pk);
-        tmem_st16(tDP + (c0 >> 1), dk);
-        // dS row segment -> shared memory, rows [c0, c0+32) = 4 chunks of 8
+        tmem_st16(tmem + lane_base + sbuf + 32 * ch + 16 * half, pk);
+      }
+      ok = mbar_wait(&ctl->dp_full, i & 1, abort, &g_device_error, kDevErrTimeoutSoftmax);
+      if (!ok) break;
+      tc_fence_after();
+      // dS = P (dP - D); dQ_{i-1} has finished reading the shared dS buffer
+      // (it was issued before dP^T_i).
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        uint32_t dr[32];
+        __syncwarp();
+        tmem_ld32(tDP + 32 * half, dr);
+        uint32_t dk[16];
+#pragma unroll
+        for (int c = 0; c < 32; c += 4) {
+          const int col = 64 * ch + 32 * half + c;
+          const float4 d4 = *reinterpret_cast<const float4*>(&a.D[col]);
+          const float ds0 = pv[32 * half + c + 0] * (__uint_as_float(dr[c + 0]) - d4.x);
+          const float ds1 = pv[32 * half + c + 1] * (__uint_as_float(dr[c + 1]) - d4.y);
+          const float ds2 = pv[32 * half + c + 2] * (__uint_as_float(dr[c + 2]) - d4.z);
+          const float ds3 = pv[32 * half + c + 3] * (__uint_as_float(dr[c + 3]) - d4.w);
+          dk[c / 2] = pack_bf16x2(ds0, ds1);
+          dk[c / 2 + 1] = pack_bf16x2(ds2, ds3);
+        }
+        // dS^T for this warp's rows -> the first 32 columns of its own dP^T
+        // column range (this warp has finished reading them).
+        __syncwarp();
+        tmem_st16(tDP + 16 * half, dk);
+        // dS -> shared memory for the dQ MMA: rows [col0, col0 + 32)
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          const int chunk = (c0 >> 3) + q;
-          *reinterpret_cast<uint4*>(sDS + ds_smem_offset(threadIdx.x, chunk)) =
+          const int chunk = ((64 * ch + 32 * half) >> 3) + q;
+          *reinterpret_cast<uint4*>(sDS + ds_smem_offset(kl, chunk)) =
               make_uint4(dk[4 * q], dk[4 * q + 1], dk[4 * q + 2], dk[4 * q + 3]);
         }
       }
-      // Generic-proxy shared-memory writes -> visible to the tensor core.
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(&ctl->p_full);
     }
-    // -------------------------------------------------- dK / dV epilogue
+    // ------------------------------------------ dK (ch 0) / dV (ch 1) epilogue
     if (ok) ok = mbar_wait(&ctl->kd_full, 0, abort, &g_device_error, kDevErrTimeoutEpilogue);
     if (ok) {
       tc_fence_after();
       uint32_t r[kHeadDim];
       __syncwarp();
-      tmem_ld64(tmem + lane_base + kBwdTmemDK, r);
+      tmem_ld64(tmem + lane_base + (ch == 0 ? kBwdTmemDK : kBwdTmemDV), r);
       if (j < geo.T) {
-        uint4* dst = reinterpret_cast<uint4*>(p.dk + (static_cast<size_t>(j) * geo.Hkv + w.g) * kHeadDim);
+        const float sc = ch == 0 ? p.scale : 1.f;
+        __nv_bfloat16* base = ch == 0 ? p.dk : p.dv;
+        uint4* dst = reinterpret_cast<uint4*>(base + (static_cast<size_t>(j) * geo.Hkv + w.g) * kHeadDim);
 #pragma unroll
         for (int i = 0; i < kHeadDim / 8; ++i) {
           uint4 v;
-          v.x = pack_bf16x2(__uint_as_float(r[8 * i + 0]) * p.scale, __uint_as_float(r[8 * i + 1]) * p.scale);
-          v.y = pack_bf16x2(__uint_as_float(r[8 * i + 2]) * p.scale, __uint_as_float(r[8 * i + 3]) * p.scale);
-          v.z = pack_bf16x2(__uint_as_float(r[8 * i + 4]) * p.scale, __uint_as_float(r[8 * i + 5]) * p.scale);
-          v.w = pack_bf16x2(__uint_as_float(r[8 * i + 6]) * p.scale, __uint_as_float(r[8 * i + 7]) * p.scale);
-          dst[i] = v;
-        }
-      }
-      __syncwarp();
-      tmem_ld64(tmem + lane_base + kBwdTmemDV, r);
-      if (j < geo.T) {
-        uint4* dst = reinterpret_cast<uint4*>(p.dv + (static_cast<size_t>(j) * geo.Hkv + w.g) * kHeadDim);
-#pragma unroll
-        for (int i = 0; i < kHeadDim / 8; ++i) {
-          uint4 v;
-          v.x = pack_bf16x2(__uint_as_float(r[8 * i + 0]), __uint_as_float(r[8 * i + 1]));
-          v.y = pack_bf16x2(__uint_as_float(r[8 * i + 2]), __uint_as_float(r[8 * i + 3]));
-          v.z = pack_bf16x2(__uint_as_float(r[8 * i + 4]), __uint_as_float(r[8 * i + 5]));
-          v.w = pack_bf16x2(__uint_as_float(r[8 * i + 6]), __uint_as_float(r[8 * i + 7]));
+          v.x = pack_bf16x2(__uint_as_float(r[8 * i + 0]) * sc, __uint_as_float(r[8 * i + 1]) * sc);
+          v.y = pack_bf16x2(__uint_as_float(r[8 * i + 2]) * sc, __uint_as_float(r[8 * i + 3]) * sc);
+          v.z = pack_bf16x2(__uint_as_float(r[8 * i + 4]) * sc, __uint_as_float(r[8 * i + 5]) * sc);
+          v.w = pack_bf16x2(__uint_as_float(r[8 * i + 6]) * sc, __uint_as_float(r[8 * i + 7]) * sc);
           dst[i] = v;
         }
       }
     }
-  } else {
-    // ---------------------- warps 6-9: per-row aux loads + dQ accumulation
-    const int r = 32 * (warp & 3) + (threadIdx.x & 31);  // TMEM lane = query row of the tile
-    const uint32_t tDQ = tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16) + kBwdTmemDQ;
-    const int hh = r & (G - 1);
-    const int h = (w.g << geo.G_log2) + hh;
-    auto load_aux = [&](int i) {
-      BwdAux& a = aux[i % kBwdStages];
-      const int t = ((w.qb0 + i) << geo.P_log2) + (r >> geo.G_log2);
-      const bool valid = t < geo.T;
-      a.lse2[r] = valid ? __ldg(p.lse + static_cast<size_t>(h) * geo.T + t) * kLog2e : INFINITY;
-      a.D[r] = valid ? __ldg(p.Dvec + static_cast<size_t>(h) * geo.T + t) : 0.f;
-      if (hh == 0) a.lo[r >> geo.G_log2] = valid ? first_key(geo, t) : 0x7fffffff;
-      mbar_arrive(&ctl->aux_full[i % kBwdStages]);
-    };
-    for (int i = 0; i < kBwdStages && i < w.nq; ++i) load_aux(i);
+  } else if (warp >= kBwdWarpDq0) {
+    // ------------------------ warps 10-13: dQ tile -> TMA reduce-add to the accumulator
+    const int lg = warp & 3;
+    const int r = 32 * lg + (threadIdx.x & 31);  // TMEM lane = query row of the tile
+    const uint32_t lane_base = static_cast<uint32_t>(32 * lg) << 16;
+    const bool leader = threadIdx.x == kBwdWarpDq0 * 32;
+    uint32_t sync_phase = 0;
     bool ok = true;
     for (int i = 0; i < w.nq; ++i) {
       ok = mbar_wait(&ctl->dq_full, i & 1, abort, &g_device_error, kDevErrTimeoutBwd);
@@ -472,25 +594,38 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tc_fence_after();
       uint32_t d[kHeadDim];
       __syncwarp();
-      tmem_ld64(tDQ, d);
+      tmem_ld64(tmem + lane_base + ((i & 1) ? kBwdTmemS1 : kBwdTmemS0) + 64, d);
       tc_fence_before();
       mbar_arrive(&ctl->dq_empty);
-      const int t = ((w.qb0 + i) << geo.P_log2) + (r >> geo.G_log2);
-      if (t < geo.T) {
-        float4* dst = reinterpret_cast<float4*>(p.dq_acc + (static_cast<size_t>(t) * geo.Hq + h) * kHeadDim);
+      // the previous reduce must have finished reading the staging buffer
+      if (leader) bulk_wait_group_read<0>();
+      ok = group_sync(&ctl->dq_sync, sync_phase, abort, kDevErrTimeoutBwd);
+      if (!ok) break;
 #pragma unroll
-        for (int c = 0; c < kHeadDim / 4; ++c)
-          atomicAdd(dst + c, make_float4(__uint_as_float(d[4 * c]), __uint_as_float(d[4 * c + 1]),
-                                         __uint_as_float(d[4 * c + 2]), __uint_as_float(d[4 * c + 3])));
+      for (int hlf = 0; hlf < 2; ++hlf) {
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const uint32_t off = static_cast<uint32_t>(hlf * 16384 + r * 128 + ((c ^ (r & 7)) << 4));
+          *reinterpret_cast<uint4*>(sDQ + off) = make_uint4(d[32 * hlf + 4 * c], d[32 * hlf + 4 * c + 1],
+                                                            d[32 * hlf + 4 * c + 2], d[32 * hlf + 4 * c + 3]);
+        }
       }
-      // Block i's aux stage is free: its P/dS pass finished before dQ_i.
-      if (i + kBwdStages < w.nq) load_aux(i + kBwdStages);
+      fence_proxy_async_smem();
+      ok = group_sync(&ctl->dq_sync, sync_phase, abort, kDevErrTimeoutBwd);
+      if (!ok) break;
+      if (leader) {
+        const int q0 = (w.qb0 + i) << geo.P_log2;
+        tma_reduce_add_3d(&tm_dq, sDQ, 0, w.g << geo.G_log2, q0);
+        tma_reduce_add_3d(&tm_dq, sDQ + 16384, 32, w.g << geo.G_log2, q0);
+        bulk_commit_group();
+      }
     }
+    if (leader) bulk_wait_group<0>();
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == kBwdWarpMma) {
     tc_fence_after();
     tmem_dealloc(tmem, kBwdTmemCols);
   }
@@ -502,18 +637,19 @@ inline sink_attn_status bwd_launch(const Geometry& geo, float scale, const void*
                                    void* dk, void* dv, float* dsinks, uint8_t* ws_base, const BwdWorkspace& ws,
                                    cudaStream_t stream, cudaEvent_t ev_main_begin, cudaEvent_t ev_main_end) {
   float* dq_acc = reinterpret_cast<float*>(ws_base + ws.dq_acc);
-  float* Dvec = reinterpret_cast<float*>(ws_base + ws.Dvec);
   float* partials = reinterpret_cast<float*>(ws_base + ws.partials);
 
   // 1. preprocess
   PreParams pp;
-  pp.T = geo.T;
-  pp.Hq = geo.Hq;
+  pp.geo = geo;
   pp.out = static_cast<const __nv_bfloat16*>(out);
   pp.dout = static_cast<const __nv_bfloat16*>(dout);
   pp.lse = lse;
   pp.sinks = sinks;
-  pp.Dvec = Dvec;
+  pp.Dvec = reinterpret_cast<float*>(ws_base + ws.Dvec);
+  pp.lse2_blk = reinterpret_cast<float*>(ws_base + ws.lse2_blk);
+  pp.D_blk = reinterpret_cast<float*>(ws_base + ws.D_blk);
+  pp.lo_blk = reinterpret_cast<int*>(ws_base + ws.lo_blk);
   pp.partials = partials;
   pp.dq_acc = dq_acc;
   pp.num_pre_blocks = ws.num_pre_blocks;
@@ -522,11 +658,12 @@ inline sink_attn_status bwd_launch(const Geometry& geo, float scale, const void*
 
   // 2. main
   const int G = 1 << geo.G_log2;
-  CUtensorMap tq, tk, tv, tdo;
+  CUtensorMap tq, tk, tv, tdo, tdq;
   if (!make_map_3d(&tq, q, kHeadDim, geo.Hq, geo.T, G, 1 << geo.P_log2) ||
       !make_map_3d(&tdo, dout, kHeadDim, geo.Hq, geo.T, G, 1 << geo.P_log2) ||
       !make_map_3d(&tk, k, kHeadDim, geo.Hkv, geo.T, 1, kBlockN) ||
-      !make_map_3d(&tv, v, kHeadDim, geo.Hkv, geo.T, 1, kBlockN))
+      !make_map_3d(&tv, v, kHeadDim, geo.Hkv, geo.T, 1, kBlockN) ||
+      !make_map_3d_f32(&tdq, dq_acc, kHeadDim, geo.Hq, geo.T, G, 1 << geo.P_log2))
     return SINK_ATTN_ERR_CUDA;
   static int smem_set = 0;
   if (!smem_set) {
@@ -539,17 +676,16 @@ inline sink_attn_status bwd_launch(const Geometry& geo, float scale, const void*
   bp.geo = geo;
   bp.scale = scale;
   bp.scale_log2 = scale * kLog2e;
-  bp.lse = lse;
-  bp.Dvec = Dvec;
-  bp.dq_acc = dq_acc;
+  bp.lse2_blk = pp.lse2_blk;
+  bp.D_blk = pp.D_blk;
+  bp.lo_blk = pp.lo_blk;
   bp.dk = static_cast<__nv_bfloat16*>(dk);
   bp.dv = static_cast<__nv_bfloat16*>(dv);
-  bp.num_key_tiles = (geo.T + kBlockN - 1) / kBlockN;
-  const int64_t grid = static_cast<int64_t>(bp.num_key_tiles) * geo.Hkv;
+  const int64_t grid = static_cast<int64_t>((geo.T + kBlockN - 1) / kBlockN) * geo.Hkv;
   if (grid > 0x7fffffff) return SINK_ATTN_ERR_UNSUPPORTED;
   if (ev_main_begin) cudaEventRecord(ev_main_begin, stream);
   sink_attn_bwd_main_kernel<<<static_cast<unsigned>(grid), kBwdThreads, kBwdSmemBytes, stream>>>(tq, tk, tv, tdo,
-                                                                                                  bp);
+                                                                                                  tdq, bp);
   if (ev_main_end) cudaEventRecord(ev_main_end, stream);
   if (cudaPeekAtLastError() != cudaSuccess) return SINK_ATTN_ERR_CUDA;
 
