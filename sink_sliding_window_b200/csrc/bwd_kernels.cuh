@@ -298,6 +298,37 @@ __device__ __forceinline__ uint32_t ds_smem_offset(int key, int chunk16) {
   return static_cast<uint32_t>(half * 16384 + (key >> 3) * 1024 + (key & 7) * 128 + ((c ^ (key & 7)) << 4));
 }
 
+// P^T for this thread's key over the 64 query rows [64*ch, 64*ch+64) of a
+// tile: P = 2^(S^T * scale*log2e - lse2), zero where the pair is masked,
+// rounded to bf16 and packed in row pairs (pk[r/2] holds rows r, r+1).
+template <bool kMask>
+__device__ __forceinline__ void bwd_p_rows(uint32_t tS, const BwdAux& a, int ch, float sl2, int j, int q0, int G_log2,
+                                           uint32_t* pk) {
+#pragma unroll
+  for (int half = 0; half < 2; ++half) {
+    uint32_t sr[32];
+    __syncwarp();
+    tmem_ld32(tS + 32 * half, sr);
+#pragma unroll
+    for (int c = 0; c < 32; c += 4) {
+      const int col = 64 * ch + 32 * half + c;
+      const float4 l4 = *reinterpret_cast<const float4*>(&a.lse2[col]);
+      const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+      float pe[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        pe[u] = ex2_approx(fmaf(__uint_as_float(sr[c + u]), sl2, -lv[u]));
+        if (kMask) {
+          const int pos = (col + u) >> G_log2;
+          if (!(j >= a.lo[pos] && j <= q0 + pos)) pe[u] = 0.f;
+        }
+      }
+      pk[16 * half + c / 2] = pack_bf16x2(pe[0], pe[1]);
+      pk[16 * half + c / 2 + 1] = pack_bf16x2(pe[2], pe[3]);
+    }
+  }
+}
+
 __global__ void __launch_bounds__(kBwdThreads, 1)
     sink_attn_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -484,42 +515,20 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                         (w.k0 >= a.lo[(kBlockM >> geo.G_log2) - 1]);
       const uint32_t tS = tmem + lane_base + sbuf + 64 * ch;
       const uint32_t tDP = tmem + lane_base + kBwdTmemDP + 64 * ch;
-      float pv[64];
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        uint32_t sr[32];
-        __syncwarp();
-        tmem_ld32(tS + 32 * half, sr);
-#pragma unroll
-        for (int c = 0; c < 32; c += 4) {
-          const int col = 64 * ch + 32 * half + c;
-          const float4 l4 = *reinterpret_cast<const float4*>(&a.lse2[col]);
-          const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            float pe = ex2_approx(fmaf(__uint_as_float(sr[c + u]), sl2, -lv[u]));
-            if (!full) {
-              const int pos = (col + u) >> geo.G_log2;
-              if (!(j >= a.lo[pos] && j <= q0 + pos)) pe = 0.f;
-            }
-            pv[32 * half + c + u] = pe;
-          }
-        }
-      }
+      uint32_t pk[32];
+      // The mask test is resolved once per tile (CTA-uniform), not per element.
+      if (full)
+        bwd_p_rows<false>(tS, a, ch, sl2, j, q0, geo.G_log2, pk);
+      else
+        bwd_p_rows<true>(tS, a, ch, sl2, j, q0, geo.G_log2, pk);
       // Both warps of this lane group have read S^T: P^T (bf16) may now
       // overwrite its first 64 columns.
       tc_fence_before();
       ok = group_sync(&ctl->pair_sync[lg], pair_phase, abort, kDevErrTimeoutSoftmax);
       if (!ok) break;
       tc_fence_after();
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        uint32_t pk[16];
-#pragma unroll
-        for (int c = 0; c < 16; ++c) pk[c] = pack_bf16x2(pv[32 * half + 2 * c], pv[32 * half + 2 * c + 1]);
-        __syncwarp();
-        tmem_st16(tmem + lane_base + sbuf + 32 * ch + 16 * half, pk);
-      }
+      __syncwarp();
+      tmem_st32(tmem + lane_base + sbuf + 32 * ch, pk);
       ok = mbar_wait(&ctl->dp_full, i & 1, abort, &g_device_error, kDevErrTimeoutSoftmax);
       if (!ok) break;
       tc_fence_after();
@@ -535,10 +544,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         for (int c = 0; c < 32; c += 4) {
           const int col = 64 * ch + 32 * half + c;
           const float4 d4 = *reinterpret_cast<const float4*>(&a.D[col]);
-          const float ds0 = pv[32 * half + c + 0] * (__uint_as_float(dr[c + 0]) - d4.x);
-          const float ds1 = pv[32 * half + c + 1] * (__uint_as_float(dr[c + 1]) - d4.y);
-          const float ds2 = pv[32 * half + c + 2] * (__uint_as_float(dr[c + 2]) - d4.z);
-          const float ds3 = pv[32 * half + c + 3] * (__uint_as_float(dr[c + 3]) - d4.w);
+          const float2 p01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&pk[16 * half + c / 2]));
+          const float2 p23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&pk[16 * half + c / 2 + 1]));
+          const float ds0 = p01.x * (__uint_as_float(dr[c + 0]) - d4.x);
+          const float ds1 = p01.y * (__uint_as_float(dr[c + 1]) - d4.y);
+          const float ds2 = p23.x * (__uint_as_float(dr[c + 2]) - d4.z);
+          const float ds3 = p23.y * (__uint_as_float(dr[c + 3]) - d4.w);
           dk[c / 2] = pack_bf16x2(ds0, ds1);
           dk[c / 2 + 1] = pack_bf16x2(ds2, ds3);
         }
