@@ -528,18 +528,19 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       if (!ok) break;
       tc_fence_after();
       __syncwarp();
-      tmem_st32(tmem + lane_base + sbuf + 32 * ch, pk);
+      tmem_st32_nowait(tmem + lane_base + sbuf + 32 * ch, pk);
       ok = mbar_wait(&ctl->dp_full, i & 1, abort, &g_device_error, kDevErrTimeoutSoftmax);
       if (!ok) break;
       tc_fence_after();
       // dS = P (dP - D); dQ_{i-1} has finished reading the shared dS buffer
       // (it was issued before dP^T_i).
+      uint32_t ds_all[32];
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
         uint32_t dr[32];
         __syncwarp();
         tmem_ld32(tDP + 32 * half, dr);
-        uint32_t dk[16];
+        uint32_t* dk = ds_all + 16 * half;
 #pragma unroll
         for (int c = 0; c < 32; c += 4) {
           const int col = 64 * ch + 32 * half + c;
@@ -556,7 +557,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         // dS^T for this warp's rows -> the first 32 columns of its own dP^T
         // column range (this warp has finished reading them).
         __syncwarp();
-        tmem_st16(tDP + 16 * half, dk);
+        tmem_st16_nowait(tDP + 16 * half, dk);
         // dS -> shared memory for the dQ MMA: rows [col0, col0 + 32)
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
@@ -565,6 +566,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
               make_uint4(dk[4 * q], dk[4 * q + 1], dk[4 * q + 2], dk[4 * q + 3]);
         }
       }
+      // P^T and dS^T stores must have landed before the MMA warp reads them
+      tmem_wait_st_keep32(pk);
+      tmem_wait_st_keep32(ds_all);
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(&ctl->p_full);

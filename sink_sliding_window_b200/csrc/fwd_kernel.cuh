@@ -100,6 +100,47 @@ __device__ __forceinline__ void fwd_issue_pv(uint32_t tmem_o, uint32_t tmem_p, u
   }
 }
 
+// One key tile of one query row: mask (kMask), row max, lazily raised
+// reference max, P = 2^(S*scale*log2e - m) packed to bf16 pairs in s[0..63],
+// and the row sum of P.  s[] holds the row's 128 fp32 logits on entry.
+struct FwdRowStep {
+  bool need;    // the reference max was raised
+  float alpha;  // factor applied to the running sum / O (1 when not raised)
+  float m_new;  // reference max after this tile
+  float sum;    // sum of this tile's P
+};
+
+template <bool kMask>
+__device__ __forceinline__ FwdRowStep fwd_row_step(uint32_t* s, int c_lo, int c_hi, float sl2, float m_ref) {
+  float x[kBlockN];
+#pragma unroll
+  for (int c = 0; c < kBlockN; ++c) {
+    x[c] = __uint_as_float(s[c]);
+    if (kMask) x[c] = (c < c_lo || c > c_hi) ? -INFINITY : x[c];
+  }
+  float mx = fmax3(x[0], x[1], x[2]);
+#pragma unroll
+  for (int c = 3; c < kBlockN - 1; c += 2) mx = fmax3(mx, x[c], x[c + 1]);
+  mx = fmaxf(mx, x[kBlockN - 1]);
+  const float mx2 = mx * sl2;
+  FwdRowStep r;
+  r.need = mx2 > m_ref + kRescaleLog2;
+  r.alpha = r.need ? ex2_approx(m_ref - mx2) : 1.f;
+  r.m_new = r.need ? mx2 : m_ref;
+  const float m_use = (r.m_new == -INFINITY) ? 0.f : r.m_new;
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int c = 0; c < kBlockN / 2; ++c) {
+    const float e0 = ex2_approx(fmaf(x[2 * c], sl2, -m_use));
+    const float e1 = ex2_approx(fmaf(x[2 * c + 1], sl2, -m_use));
+    acc[(2 * c) & 3] += e0;
+    acc[(2 * c + 1) & 3] += e1;
+    s[c] = pack_bf16x2(e0, e1);
+  }
+  r.sum = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+  return r;
+}
+
 __global__ void __launch_bounds__(kFwdThreads, 2)
     sink_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                          const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
@@ -216,39 +257,19 @@ __global__ void __launch_bounds__(kFwdThreads, 2)
       uint32_t sr[kBlockN];
       tmem_ld64(tS, sr);
       tmem_ld64(tS + 64, sr + 64);
-      float x[kBlockN];
-#pragma unroll
-      for (int c = 0; c < kBlockN; ++c) x[c] = __uint_as_float(sr[c]);
       const int ts = w.kv_lo + j * kBlockN;
-      // CTA-uniform: does any row of this tile see a masked key?
-      if (ts + kBlockN - 1 > w.t0 || ts < w.lo_max) {
-        const int c_lo = lo_r - ts, c_hi = hi_r - ts;
-#pragma unroll
-        for (int c = 0; c < kBlockN; ++c) x[c] = (c < c_lo || c > c_hi) ? -INFINITY : x[c];
-      }
-      float mx = x[0];
-#pragma unroll
-      for (int c = 1; c < kBlockN; ++c) mx = fmaxf(mx, x[c]);
-      const float mx2 = mx * sl2;
-      const bool need = mx2 > m_ref + kRescaleLog2;
-      float alpha = 1.f;
-      if (need) {
-        alpha = ex2_approx(m_ref - mx2);
-        l *= alpha;
-      }
-      const float m_new = need ? mx2 : m_ref;
-      const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
-      float sum0 = 0.f, sum1 = 0.f;
-      uint32_t pk[kBlockN / 2];
-#pragma unroll
-      for (int c = 0; c < kBlockN / 2; ++c) {
-        const float e0 = ex2_approx(fmaf(x[2 * c], sl2, -m_use));
-        const float e1 = ex2_approx(fmaf(x[2 * c + 1], sl2, -m_use));
-        sum0 += e0;
-        sum1 += e1;
-        pk[c] = pack_bf16x2(e0, e1);
-      }
-      l += sum0 + sum1;
+      // CTA-uniform: does any row of this tile see a masked key?  Resolved
+      // once per tile, not per element.
+      FwdRowStep st;
+      if (ts + kBlockN - 1 > w.t0 || ts < w.lo_max)
+        st = fwd_row_step<true>(sr, lo_r - ts, hi_r - ts, sl2, m_ref);
+      else
+        st = fwd_row_step<false>(sr, 0, 0, sl2, m_ref);
+      const bool need = st.need;
+      const float alpha = st.alpha;
+      const float m_new = st.m_new;
+      l = l * alpha + st.sum;
+      uint32_t* pk = sr;  // fwd_row_step packed P (bf16 pairs) into sr[0..63]
       __syncwarp();
       tmem_st32(tS, pk);
       tmem_st32(tS + 32, pk + 32);
