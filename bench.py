@@ -196,6 +196,24 @@ def measured_traffic():
     return t.get("dram_bytes_per_launch") if t.get("kernel_source_hash") == kernel_source_hash() else None
 
 
+# ----------------------------------------------------------- aggregation
+def max_over_ranks(x, dist, device):
+    """Largest value of x over all ranks (the slowest rank's time); x itself
+    when running alone."""
+    if dist is None:
+        return float(x)
+    import torch
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world, flops_per_step, steps, ms):
+    """Whole-job TFLOP/s: every rank runs its own replica of the step, so the
+    job does world x steps steps in the slowest rank's time."""
+    return world * flops_per_step * steps / (ms / 1e3) / 1e12
+
+
 # ------------------------------------------------------------------- arms
 def run_reference(args, rank):
     if rank != 0:
@@ -203,7 +221,7 @@ def run_reference(args, rank):
     # Size each step so that all warmup + timed steps take about two minutes:
     # the sample's work grows ~linearly with the window-layer prefix and
     # quadratically with the full-causal prefix.
-    budget = 120.0 / (args.warmup + args.steps)
+    budget = args.budget_s / (args.warmup + args.steps)
     secs1, _, _, _ = oracle_sample(256, 256)  # calibration, untimed
     lw, lf = 256, 256
     while lw < S and secs1 * (2 * lw / 256 + (lf / 256) ** 2) / 3 * 2 < budget:
@@ -300,13 +318,10 @@ def run_ours(args, rank, world, torch, dist):
     kern_ms = float(np.mean([b.elapsed_time(e) for b, e in prof]))
     if ops.device_error() != 0:
         raise RuntimeError("a kernel reported a timed-out wait")
-    if dist is not None:
-        t = torch.tensor([ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms, dist, "cuda")
 
     flops = step_flops()
-    value = world * flops * args.steps / (ms / 1e3) / 1e12
+    value = job_throughput(world, flops, args.steps, ms)
     launches = args.steps * len(LAYERS) * (ops.fwd_launches(T, HQ, HKV, D, B, S) + ops.bwd_launches(T, HQ, HKV, D, B, S))
 
     # ---- end to end through host buffers (pinned), copies inside the region
@@ -332,12 +347,8 @@ def run_ours(args, rank, world, torch, dist):
     x1.record(stream)
     torch.cuda.synchronize()
     barrier()
-    e2e_ms = x0.elapsed_time(x1)
-    if dist is not None:
-        t = torch.tensor([e2e_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_value = world * flops * e2e_steps / (e2e_ms / 1e3) / 1e12
+    e2e_ms = max_over_ranks(x0.elapsed_time(x1), dist, "cuda")
+    e2e_value = job_throughput(world, flops, e2e_steps, e2e_ms)
 
     if rank != 0:
         return
@@ -360,7 +371,7 @@ def run_ours(args, rank, world, torch, dist):
         "clocks": clk,
     }
     if world == 1 and not args.skip_cpu_baseline:
-        secs, cflops, desc, threads = oracle_sample()
+        secs, cflops, desc, threads = oracle_sample(S, 2048)
         line["cpu_baseline"] = {"value": cflops / secs / 1e12, "unit": "TFLOP/s", "cores": threads,
                                 "kind": "oracle", "sample": desc, "seconds": secs}
     print(json.dumps(line), flush=True)
@@ -374,6 +385,8 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--skip-cpu-baseline", action="store_true")
+    ap.add_argument("--budget-s", type=float, default=120.0,
+                    help="--impl reference: seconds all warmup + timed oracle steps should take")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

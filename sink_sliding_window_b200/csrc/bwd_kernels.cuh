@@ -99,50 +99,62 @@ __device__ __forceinline__ float dot8_bf16(uint4 a, uint4 b) {
   return s;
 }
 
-// Grid (num_pre_blocks, Hq); thread = one token (padded up to whole query
-// tiles) of head blockIdx.y.
+// Grid (num_pre_blocks, Hq).  Each group of 8 lanes reads one 128-byte row
+// (token, head blockIdx.y) of out and dout with one 16-byte load per lane, so
+// a warp-wide load covers 4 rows; a CTA covers kPreThreads tokens (padded up
+// to whole query tiles).
 __global__ void __launch_bounds__(kPreThreads) sink_attn_bwd_preprocess_kernel(const PreParams p) {
   __shared__ float warp_sums[kPreThreads / 32];
   const Geometry& geo = p.geo;
   const int h = blockIdx.y;
-  const int t = blockIdx.x * kPreThreads + threadIdx.x;
   const int t_pad = geo.num_qblocks << geo.P_log2;
-  float contrib = 0.f;
-  if (t < t_pad) {
-    const int qb = t >> geo.P_log2;
-    const int pos = t & ((1 << geo.P_log2) - 1);
-    const int g = h >> geo.G_log2;
-    const int r = (pos << geo.G_log2) + (h & ((1 << geo.G_log2) - 1));
-    const size_t bi = (static_cast<size_t>(qb) * geo.Hkv + g) * kBlockM + r;
+  const int lane = threadIdx.x & 31;
+  const int sub = lane & 7;              // 16-byte piece of the row
+  const int t_base = blockIdx.x * kPreThreads + (threadIdx.x >> 5) * 32;  // this warp's 32 tokens
+  float contrib = 0.f;                   // valid in lanes with sub == 0
+#pragma unroll 2
+  for (int it = 0; it < 8; ++it) {
+    const int t = t_base + it * 4 + (lane >> 3);
+    float D = 0.f;
     if (t < geo.T) {
       const size_t row = (static_cast<size_t>(t) * geo.Hq + h) * kHeadDim;
-      const uint4* o = reinterpret_cast<const uint4*>(p.out + row);
-      const uint4* gr = reinterpret_cast<const uint4*>(p.dout + row);
-      float D = 0.f;
-#pragma unroll
-      for (int i = 0; i < kHeadDim / 8; ++i) D += dot8_bf16(__ldg(o + i), __ldg(gr + i));
-      const float lse = __ldg(p.lse + static_cast<size_t>(h) * geo.T + t);
-      p.Dvec[static_cast<size_t>(h) * geo.T + t] = D;
-      p.D_blk[bi] = D;
-      p.lse2_blk[bi] = lse * kLog2e;
-      const float psink = ex2_approx((__ldg(p.sinks + h) - lse) * kLog2e);  // e^{s_h - lse}; 0 for s = -inf
-      contrib = -psink * D;
-      float4* acc = reinterpret_cast<float4*>(p.dq_acc + row);
-#pragma unroll
-      for (int i = 0; i < kHeadDim / 4; ++i) acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (h == 0) p.lo_blk[static_cast<size_t>(qb) * kBlockM + pos] = first_key(geo, t);
-    } else {
-      // padding rows of the last query tile: P = 0 and dS = 0 there
-      p.D_blk[bi] = 0.f;
-      p.lse2_blk[bi] = INFINITY;
-      if (h == 0) p.lo_blk[static_cast<size_t>(qb) * kBlockM + pos] = 0x7fffffff;
+      D = dot8_bf16(__ldg(reinterpret_cast<const uint4*>(p.out + row) + sub),
+                    __ldg(reinterpret_cast<const uint4*>(p.dout + row) + sub));
+      float4* acc = reinterpret_cast<float4*>(p.dq_acc + row) + 2 * sub;
+      acc[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+      acc[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    // sum the 8 pieces of the row (fixed butterfly)
+    D += __shfl_xor_sync(0xffffffffu, D, 1);
+    D += __shfl_xor_sync(0xffffffffu, D, 2);
+    D += __shfl_xor_sync(0xffffffffu, D, 4);
+    if (sub == 0 && t < t_pad) {
+      const int qb = t >> geo.P_log2;
+      const int pos = t & ((1 << geo.P_log2) - 1);
+      const int g = h >> geo.G_log2;
+      const int r = (pos << geo.G_log2) + (h & ((1 << geo.G_log2) - 1));
+      const size_t bi = (static_cast<size_t>(qb) * geo.Hkv + g) * kBlockM + r;
+      if (t < geo.T) {
+        const float lse = __ldg(p.lse + static_cast<size_t>(h) * geo.T + t);
+        p.Dvec[static_cast<size_t>(h) * geo.T + t] = D;
+        p.D_blk[bi] = D;
+        p.lse2_blk[bi] = lse * kLog2e;
+        const float psink = ex2_approx((__ldg(p.sinks + h) - lse) * kLog2e);  // e^{s_h - lse}; 0 for s = -inf
+        contrib -= psink * D;
+        if (h == 0) p.lo_blk[static_cast<size_t>(qb) * kBlockM + pos] = first_key(geo, t);
+      } else {
+        // padding rows of the last query tile: P = 0 and dS = 0 there
+        p.D_blk[bi] = 0.f;
+        p.lse2_blk[bi] = INFINITY;
+        if (h == 0) p.lo_blk[static_cast<size_t>(qb) * kBlockM + pos] = 0x7fffffff;
+      }
     }
   }
   // Fixed-order block reduction: butterfly within each warp, then warps in
   // index order.
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) contrib += __shfl_xor_sync(0xffffffffu, contrib, off);
-  if ((threadIdx.x & 31) == 0) warp_sums[threadIdx.x >> 5] = contrib;
+  if (lane == 0) warp_sums[threadIdx.x >> 5] = contrib;
   __syncthreads();
   if (threadIdx.x == 0) {
     float s = 0.f;
@@ -266,7 +278,7 @@ __device__ __forceinline__ int doc_end(const Geometry& g, int t) {
 }
 
 struct BwdTile {
-  int g, k0, qb0, nq;
+  int g, k0, qb_last, nq;  // query tiles qb_last, qb_last-1, ..., qb_last-nq+1
 };
 
 __device__ __forceinline__ BwdTile bwd_tile(const Geometry& geo) {
@@ -284,8 +296,12 @@ __device__ __forceinline__ BwdTile bwd_tile(const Geometry& geo) {
   const int k_last = min(w.k0 + kBlockN - 1, geo.T - 1);
   int q_hi = doc_end(geo, k_last) - 1;
   if (geo.window > 0) q_hi = min(q_hi, k_last + geo.window - 1);
-  w.qb0 = w.k0 >> geo.P_log2;
-  w.nq = (q_hi >> geo.P_log2) - w.qb0 + 1;
+  // Visit query tiles from the last one down: the key tiles of a document
+  // that run at the same time then add into the same rows of the fp32 dq
+  // accumulator at about the same time, and those rows stay in L2.
+  const int qb0 = w.k0 >> geo.P_log2;
+  w.qb_last = q_hi >> geo.P_log2;
+  w.nq = w.qb_last - qb0 + 1;
   return w;
 }
 
@@ -389,7 +405,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             !mbar_wait(&ctl->qdo_empty[s], ((i / kBwdStages) - 1) & 1, abort, &g_device_error,
                        kDevErrTimeoutProducer))
           break;
-        const int qb = w.qb0 + i;
+        const int qb = w.qb_last - i;
         const int q0 = qb << geo.P_log2;
         const size_t blk = (static_cast<size_t>(qb) * geo.Hkv + w.g) * kBlockM;
         mbar_arrive_expect_tx(&ctl->qdo_full[s], 2 * kTileBytes + 3 * kBlockM * 4);
@@ -508,7 +524,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       if (!ok) break;
       tc_fence_after();
       const BwdAux& a = aux[st];
-      const int q0 = (w.qb0 + i) << geo.P_log2;
+      const int q0 = (w.qb_last - i) << geo.P_log2;
       const int q_last = q0 + (1 << geo.P_log2) - 1;
       // CTA-uniform: is every (key, row) pair of this tile allowed?
       const bool full = (w.k0 + kBlockN - 1 < geo.T) && (q_last < geo.T) && (w.k0 + kBlockN - 1 <= q0) &&
@@ -629,7 +645,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       ok = group_sync(&ctl->dq_sync, sync_phase, abort, kDevErrTimeoutBwd);
       if (!ok) break;
       if (leader) {
-        const int q0 = (w.qb0 + i) << geo.P_log2;
+        const int q0 = (w.qb_last - i) << geo.P_log2;
         tma_reduce_add_3d(&tm_dq, sDQ, 0, w.g << geo.G_log2, q0);
         tma_reduce_add_3d(&tm_dq, sDQ + 16384, 32, w.g << geo.G_log2, q0);
         bulk_commit_group();
