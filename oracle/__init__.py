@@ -54,9 +54,14 @@ def _bind(path):
     lib.oracle_fwd_rows_bf16.argtypes = common + [P, P, P, P, I, Dbl, P, I64, P, P, I]
     lib.oracle_bwd_f64.argtypes = common + [P, P, P, P, I, Dbl, P, P, P, P, P, P, I]
     lib.oracle_bwd_bf16.argtypes = common + [P, P, P, P, I, Dbl, P, P, P, P, P, P, I]
+    lib.oracle_bwd_dq_rows_f64.argtypes = common + [P, P, P, P, I, Dbl, P, P, P, I64, P, I]
+    lib.oracle_bwd_dq_rows_bf16.argtypes = common + [P, P, P, P, I, Dbl, P, P, P, I64, P, I]
+    lib.oracle_bwd_dkv_rows_f64.argtypes = common + [P, P, P, P, I, Dbl, P, P, P, I64, P, P, I]
+    lib.oracle_bwd_dkv_rows_bf16.argtypes = common + [P, P, P, P, I, Dbl, P, P, P, I64, P, P, I]
     lib.oracle_bf16_to_f64.argtypes = [P, P, I64]
     for f in ("oracle_fwd_f64", "oracle_fwd_bf16", "oracle_fwd_rows_f64", "oracle_fwd_rows_bf16",
-              "oracle_bwd_f64", "oracle_bwd_bf16", "oracle_bf16_to_f64", "oracle_max_threads"):
+              "oracle_bwd_f64", "oracle_bwd_bf16", "oracle_bwd_dq_rows_f64", "oracle_bwd_dq_rows_bf16",
+              "oracle_bwd_dkv_rows_f64", "oracle_bwd_dkv_rows_bf16", "oracle_bf16_to_f64", "oracle_max_threads"):
         getattr(lib, f).restype = I
     return lib
 
@@ -149,6 +154,49 @@ class Oracle:
         _check(rc, "oracle bwd")
         return dq, dk, dv, ds
 
+    def _bwd_args(self, q, k, v, sinks, dout, out_for_D):
+        if _is_bf16_bits(q):
+            conv, sconv, sfx = np.uint16, np.float32, "bf16"
+        else:
+            conv, sconv, sfx = np.float64, np.float64, "f64"
+        args = [np.ascontiguousarray(x, conv) for x in (q, k, v)]
+        s = np.ascontiguousarray(sinks, sconv)
+        o = None if out_for_D is None else np.ascontiguousarray(out_for_D, conv)
+        do = np.ascontiguousarray(dout, conv)
+        return args, s, o, do, sfx
+
+    def bwd_dq_rows(self, q, k, v, sinks, cu_seqlens, window, scale, dout, rows, out_for_D=None, nthreads=0):
+        """dq of the backward definition for the query tokens ``rows`` (every
+        head).  Returns dq_rows [n, Hq, D] float64."""
+        T, Hq, D = q.shape
+        Hkv = k.shape[1]
+        cu = _cu(cu_seqlens, T)
+        r = np.ascontiguousarray(rows, np.int64)
+        out = np.empty((r.shape[0], Hq, D), np.float64)
+        args, s, o, do, sfx = self._bwd_args(q, k, v, sinks, dout, out_for_D)
+        fn = getattr(self.lib, f"oracle_bwd_dq_rows_{sfx}")
+        rc = fn(T, Hq, Hkv, D, cu.shape[0] - 1, _ptr(cu), *map(_ptr, args), _ptr(s), int(window), float(scale),
+                _ptr(o), _ptr(do), _ptr(r), r.shape[0], _ptr(out), int(nthreads))
+        _check(rc, "oracle bwd_dq_rows")
+        return out
+
+    def bwd_dkv_rows(self, q, k, v, sinks, cu_seqlens, window, scale, dout, keys, out_for_D=None, nthreads=0):
+        """dk and dv of the backward definition for the key tokens ``keys``
+        (sorted ascending; every key/value head).  Returns (dk_rows, dv_rows),
+        each [n, Hkv, D] float64."""
+        T, Hq, D = q.shape
+        Hkv = k.shape[1]
+        cu = _cu(cu_seqlens, T)
+        kk = np.ascontiguousarray(keys, np.int64)
+        dk = np.empty((kk.shape[0], Hkv, D), np.float64)
+        dv = np.empty((kk.shape[0], Hkv, D), np.float64)
+        args, s, o, do, sfx = self._bwd_args(q, k, v, sinks, dout, out_for_D)
+        fn = getattr(self.lib, f"oracle_bwd_dkv_rows_{sfx}")
+        rc = fn(T, Hq, Hkv, D, cu.shape[0] - 1, _ptr(cu), *map(_ptr, args), _ptr(s), int(window), float(scale),
+                _ptr(o), _ptr(do), _ptr(kk), kk.shape[0], _ptr(dk), _ptr(dv), int(nthreads))
+        _check(rc, "oracle bwd_dkv_rows")
+        return dk, dv
+
     def bf16_bits_to_f64(self, a):
         """Exact widening of bf16 bit patterns (uint16) to float64."""
         a = np.ascontiguousarray(a, np.uint16)
@@ -198,6 +246,14 @@ def fwd_rows(*a, **kw):
 
 def bwd(*a, **kw):
     return default().bwd(*a, **kw)
+
+
+def bwd_dq_rows(*a, **kw):
+    return default().bwd_dq_rows(*a, **kw)
+
+
+def bwd_dkv_rows(*a, **kw):
+    return default().bwd_dkv_rows(*a, **kw)
 
 
 def bf16_bits_to_f64(a):

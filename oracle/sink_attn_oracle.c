@@ -296,6 +296,166 @@ int oracle_bwd_f64(int T, int Hq, int Hkv, int D, int B, const int32_t* cu_seqle
     return err;
 }
 
+/* Backward restricted to chosen query tokens: dq for every head of each
+ * token in `rows` (fp64 inputs).  dq_i only needs row i's own probabilities,
+ * so each row is the definition above evaluated for that row alone.
+ * out_for_D as for oracle_bwd_f64.  dq_rows[n][Hq][D]. */
+int oracle_bwd_dq_rows_f64(int T, int Hq, int Hkv, int D, int B, const int32_t* cu_seqlens,
+                           const double* q, const double* k, const double* v, const double* sinks,
+                           int window, double scale, const double* out_for_D, const double* dout,
+                           const int64_t* rows, int64_t nrows, double* dq_rows, int nthreads) {
+    if (!check_common(T, Hq, Hkv, D, B, cu_seqlens) || !sinks || !rows || nrows < 0) return ORACLE_ERR_ARG;
+    if (nrows > 0 && (!q || !k || !v || !dout || !dq_rows)) return ORACLE_ERR_ARG;
+    for (int64_t r = 0; r < nrows; ++r)
+        if (rows[r] < 0 || rows[r] >= T) return ORACLE_ERR_ARG;
+    const int G = Hq / Hkv;
+    int64_t maxlen = 0;
+    for (int b = 0; b < B; ++b)
+        if (cu_seqlens[b + 1] - cu_seqlens[b] > maxlen) maxlen = cu_seqlens[b + 1] - cu_seqlens[b];
+    int err = ORACLE_OK;
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#endif
+#pragma omp parallel
+    {
+        double* logits = (double*)malloc(sizeof(double) * (size_t)(maxlen > 0 ? maxlen : 1));
+        double* orow = (double*)malloc(sizeof(double) * (size_t)D);
+        if (!logits || !orow) {
+#pragma omp atomic write
+            err = ORACLE_ERR_NOMEM;
+        } else {
+#pragma omp for schedule(dynamic, 1)
+            for (int64_t idx = 0; idx < nrows * Hq; ++idx) {
+                int64_t r = idx / Hq;
+                int h = (int)(idx % Hq);
+                int g = h / G;
+                int64_t t = rows[r];
+                int64_t a = cu_seqlens[doc_of(cu_seqlens, B, t)];
+                double lse = fwd_row(t, h, a, Hq, Hkv, D, q, k, v, sinks[h], window, scale, logits, orow);
+                const double* o = out_for_D ? out_for_D + (t * Hq + h) * (int64_t)D : orow;
+                const double* doi = dout + (t * Hq + h) * (int64_t)D;
+                double* dqi = dq_rows + (r * Hq + h) * (int64_t)D;
+                double Di = 0.0;
+                for (int d = 0; d < D; ++d) Di += doi[d] * o[d];
+                for (int d = 0; d < D; ++d) dqi[d] = 0.0;
+                int64_t j0 = first_key(t, a, window);
+                for (int64_t j = j0; j <= t; ++j) {
+                    const double* kj = k + (j * Hkv + g) * (int64_t)D;
+                    const double* vj = v + (j * Hkv + g) * (int64_t)D;
+                    double P = exp(logits[j - j0] - lse);
+                    double dP = 0.0;
+                    for (int d = 0; d < D; ++d) dP += doi[d] * vj[d];
+                    double dS = P * (dP - Di);
+                    for (int d = 0; d < D; ++d) dqi[d] += scale * dS * kj[d];
+                }
+            }
+        }
+        free(logits);
+        free(orow);
+    }
+    return err;
+}
+
+/* Backward restricted to chosen key tokens: dk and dv for every key/value
+ * head of each token in `keys` (fp64 inputs).  dk_j and dv_j sum over every
+ * query row (and every head of the group) allowed to see key j; those rows'
+ * lse_i and D_i come from their own forward rows.  keys must be sorted
+ * ascending.  dk_rows/dv_rows [n][Hkv][D]. */
+int oracle_bwd_dkv_rows_f64(int T, int Hq, int Hkv, int D, int B, const int32_t* cu_seqlens,
+                            const double* q, const double* k, const double* v, const double* sinks,
+                            int window, double scale, const double* out_for_D, const double* dout,
+                            const int64_t* keys, int64_t nkeys, double* dk_rows, double* dv_rows, int nthreads) {
+    if (!check_common(T, Hq, Hkv, D, B, cu_seqlens) || !sinks || !keys || nkeys < 0) return ORACLE_ERR_ARG;
+    if (nkeys > 0 && (!q || !k || !v || !dout || !dk_rows || !dv_rows)) return ORACLE_ERR_ARG;
+    for (int64_t r = 0; r < nkeys; ++r)
+        if (keys[r] < 0 || keys[r] >= T || (r > 0 && keys[r] < keys[r - 1])) return ORACLE_ERR_ARG;
+    if (nkeys == 0) return ORACLE_OK;
+    const int G = Hq / Hkv;
+    int64_t maxlen = 0;
+    for (int b = 0; b < B; ++b)
+        if (cu_seqlens[b + 1] - cu_seqlens[b] > maxlen) maxlen = cu_seqlens[b + 1] - cu_seqlens[b];
+    /* Query tokens that see at least one chosen key: a query t sees key j
+     * when j <= t, they share a document, and t - j < window (if any). */
+    char* need = (char*)calloc((size_t)(T > 0 ? T : 1), 1);
+    double* lse_all = (double*)malloc(sizeof(double) * (size_t)(T > 0 ? T : 1) * Hq);
+    double* D_all = (double*)malloc(sizeof(double) * (size_t)(T > 0 ? T : 1) * Hq);
+    if (!need || !lse_all || !D_all) {
+        free(need); free(lse_all); free(D_all);
+        return ORACLE_ERR_NOMEM;
+    }
+    for (int64_t r = 0; r < nkeys; ++r) {
+        int64_t j = keys[r];
+        int64_t e = cu_seqlens[doc_of(cu_seqlens, B, j) + 1];
+        int64_t hi = (window > 0 && j + window < e) ? j + window : e;
+        for (int64_t t = j; t < hi; ++t) need[t] = 1;
+    }
+    int err = ORACLE_OK;
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#endif
+    /* Pass 1: lse_i and D_i of every needed (query, head) row. */
+#pragma omp parallel
+    {
+        double* logits = (double*)malloc(sizeof(double) * (size_t)(maxlen > 0 ? maxlen : 1));
+        double* orow = (double*)malloc(sizeof(double) * (size_t)D);
+        if (!logits || !orow) {
+#pragma omp atomic write
+            err = ORACLE_ERR_NOMEM;
+        } else {
+#pragma omp for schedule(dynamic, 16)
+            for (int64_t idx = 0; idx < (int64_t)T * Hq; ++idx) {
+                int64_t t = idx / Hq;
+                int h = (int)(idx % Hq);
+                if (!need[t]) continue;
+                int64_t a = cu_seqlens[doc_of(cu_seqlens, B, t)];
+                double lse = fwd_row(t, h, a, Hq, Hkv, D, q, k, v, sinks[h], window, scale, logits, orow);
+                const double* o = out_for_D ? out_for_D + (t * Hq + h) * (int64_t)D : orow;
+                const double* doi = dout + (t * Hq + h) * (int64_t)D;
+                double Di = 0.0;
+                for (int d = 0; d < D; ++d) Di += doi[d] * o[d];
+                lse_all[t * Hq + h] = lse;
+                D_all[t * Hq + h] = Di;
+            }
+        }
+        free(logits);
+        free(orow);
+    }
+    /* Pass 2: each chosen key sums over its query rows in ascending order. */
+    if (err == ORACLE_OK) {
+#pragma omp parallel for schedule(dynamic, 1)
+        for (int64_t idx = 0; idx < nkeys * Hkv; ++idx) {
+            int64_t r = idx / Hkv;
+            int g = (int)(idx % Hkv);
+            int64_t j = keys[r];
+            int64_t e = cu_seqlens[doc_of(cu_seqlens, B, j) + 1];
+            int64_t hi = (window > 0 && j + window < e) ? j + window : e;
+            const double* kj = k + (j * Hkv + g) * (int64_t)D;
+            const double* vj = v + (j * Hkv + g) * (int64_t)D;
+            double* dkj = dk_rows + (r * Hkv + g) * (int64_t)D;
+            double* dvj = dv_rows + (r * Hkv + g) * (int64_t)D;
+            for (int d = 0; d < D; ++d) dkj[d] = dvj[d] = 0.0;
+            for (int64_t t = j; t < hi; ++t) {
+                for (int hh = 0; hh < G; ++hh) {
+                    int h = g * G + hh;
+                    const double* qi = q + (t * Hq + h) * (int64_t)D;
+                    const double* doi = dout + (t * Hq + h) * (int64_t)D;
+                    double dot = 0.0, dP = 0.0;
+                    for (int d = 0; d < D; ++d) dot += qi[d] * kj[d];
+                    for (int d = 0; d < D; ++d) dP += doi[d] * vj[d];
+                    double P = exp(scale * dot - lse_all[t * Hq + h]);
+                    double dS = P * (dP - D_all[t * Hq + h]);
+                    for (int d = 0; d < D; ++d) {
+                        dkj[d] += scale * dS * qi[d];
+                        dvj[d] += P * doi[d];
+                    }
+                }
+            }
+        }
+    }
+    free(need); free(lse_all); free(D_all);
+    return err;
+}
+
 /* bf16-input wrappers: widen exactly, then run the fp64 definition. */
 static double* widen(const uint16_t* src, int64_t n) {
     double* d = (double*)malloc(sizeof(double) * (size_t)(n > 0 ? n : 1));
@@ -362,6 +522,46 @@ int oracle_bwd_bf16(int T, int Hq, int Hkv, int D, int B, const int32_t* cu_seql
     if (qd && kd && vd && dod && sd && (od || !out_for_D_bf16))
         rc = oracle_bwd_f64(T, Hq, Hkv, D, B, cu_seqlens, qd, kd, vd, sd, window, scale, od, dod, dq, dk, dv,
                             dsinks, nthreads);
+    free(qd); free(kd); free(vd); free(dod); free(od); free(sd);
+    return rc;
+}
+
+int oracle_bwd_dq_rows_bf16(int T, int Hq, int Hkv, int D, int B, const int32_t* cu_seqlens,
+                            const uint16_t* q, const uint16_t* k, const uint16_t* v, const float* sinks,
+                            int window, double scale, const uint16_t* out_for_D_bf16, const uint16_t* dout,
+                            const int64_t* rows, int64_t nrows, double* dq_rows, int nthreads) {
+    if (T < 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || !sinks) return ORACLE_ERR_ARG;
+    if (T > 0 && (!q || !k || !v || !dout)) return ORACLE_ERR_ARG;
+    double* qd = widen(q, (int64_t)T * Hq * D);
+    double* kd = widen(k, (int64_t)T * Hkv * D);
+    double* vd = widen(v, (int64_t)T * Hkv * D);
+    double* dod = widen(dout, (int64_t)T * Hq * D);
+    double* od = out_for_D_bf16 ? widen(out_for_D_bf16, (int64_t)T * Hq * D) : NULL;
+    double* sd = widen_f32(sinks, Hq);
+    int rc = ORACLE_ERR_NOMEM;
+    if (qd && kd && vd && dod && sd && (od || !out_for_D_bf16))
+        rc = oracle_bwd_dq_rows_f64(T, Hq, Hkv, D, B, cu_seqlens, qd, kd, vd, sd, window, scale, od, dod, rows,
+                                    nrows, dq_rows, nthreads);
+    free(qd); free(kd); free(vd); free(dod); free(od); free(sd);
+    return rc;
+}
+
+int oracle_bwd_dkv_rows_bf16(int T, int Hq, int Hkv, int D, int B, const int32_t* cu_seqlens,
+                             const uint16_t* q, const uint16_t* k, const uint16_t* v, const float* sinks,
+                             int window, double scale, const uint16_t* out_for_D_bf16, const uint16_t* dout,
+                             const int64_t* keys, int64_t nkeys, double* dk_rows, double* dv_rows, int nthreads) {
+    if (T < 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || !sinks) return ORACLE_ERR_ARG;
+    if (T > 0 && (!q || !k || !v || !dout)) return ORACLE_ERR_ARG;
+    double* qd = widen(q, (int64_t)T * Hq * D);
+    double* kd = widen(k, (int64_t)T * Hkv * D);
+    double* vd = widen(v, (int64_t)T * Hkv * D);
+    double* dod = widen(dout, (int64_t)T * Hq * D);
+    double* od = out_for_D_bf16 ? widen(out_for_D_bf16, (int64_t)T * Hq * D) : NULL;
+    double* sd = widen_f32(sinks, Hq);
+    int rc = ORACLE_ERR_NOMEM;
+    if (qd && kd && vd && dod && sd && (od || !out_for_D_bf16))
+        rc = oracle_bwd_dkv_rows_f64(T, Hq, Hkv, D, B, cu_seqlens, qd, kd, vd, sd, window, scale, od, dod, keys,
+                                     nkeys, dk_rows, dv_rows, nthreads);
     free(qd); free(kd); free(vd); free(dod); free(od); free(sd);
     return rc;
 }

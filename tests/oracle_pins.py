@@ -344,6 +344,21 @@ def pin_bf16_widening(O):
     assert all(np.array_equal(x, y) for x, y in zip(ga, gb)), "bf16 widening bwd"
 
 
+def pin_restricted_backward(O):
+    """dq for chosen query tokens and dk/dv for chosen key tokens equal the
+    matching rows of the full backward (same sums, same order)."""
+    for n, (cu, W) in enumerate([([0, 40], 0), ([0, 40], 6), ([0, 9, 10, 40], 0), ([0, 9, 10, 40], 5)]):
+        q, k, v, s, cu = rand_problem(70 + n, 40, 4, 2, 8, cu=cu)
+        dout = np.random.default_rng(80 + n).standard_normal(q.shape)
+        dq, dk, dv, _ = O.bwd(q, k, v, s, cu, W, 0.25, dout)
+        rows = np.array([0, 3, 9, 10, 25, 39])
+        assert_close(O.bwd_dq_rows(q, k, v, s, cu, W, 0.25, dout, rows), dq[rows], 1e-12, f"dq rows case {n}")
+        keys = np.array([0, 8, 9, 10, 30, 39])
+        rk, rv = O.bwd_dkv_rows(q, k, v, s, cu, W, 0.25, dout, keys)
+        assert_close(rk, dk[keys], 1e-12, f"dk rows case {n}")
+        assert_close(rv, dv[keys], 1e-12, f"dv rows case {n}")
+
+
 ALL_PINS = [
     pin_library_special_case,
     pin_no_sink_is_causal_sdpa,
@@ -357,4 +372,5 @@ ALL_PINS = [
     pin_structure,
     pin_rows_match_full,
     pin_bf16_widening,
+    pin_restricted_backward,
 ]
