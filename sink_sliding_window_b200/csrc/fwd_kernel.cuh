@@ -8,30 +8,48 @@
 // tile in exactly this row order.  Every key/value tile that is loaded serves
 // all G heads of the group.
 //
-// Per key/value tile j (128 keys starting at kv_lo + 128 j):
-//   S = Q K_j^T            tcgen05.mma, bf16 in, fp32 in TMEM (128 cols)
+// Keys are consumed in steps of 64 ("halves" of a 128-key K/V tile):
+//   S_h = Q K_h^T          tcgen05.mma, bf16 in, fp32 in TMEM (64 columns),
+//                          into S/P buffer h % 2
 //   softmax (1 thread = 1 row, the row lives in that thread's TMEM lane):
 //     masked logits -> running reference max m (seeded with the sink logit,
 //     lazily raised), P = 2^(S*scale*log2e - m) as bf16 written back into the
-//     S columns, row sum l (seeded with the sink's e^{s-m} = 1)
-//   O += P V_j             tcgen05.mma with A = P from TMEM, fp32 O in TMEM
+//     buffer's first 32 columns, row sum l (seeded with the sink's e^{s-m}=1)
+//   O += P_h V_h           tcgen05.mma with A = P from TMEM, fp32 O in TMEM
+// The steps alternate between two softmax warpgroups: warpgroup b takes the
+// steps h with h % 2 == b, owns S/P buffer b and its own accumulator O_b, and
+// keeps its own running max and sum.  Softmax is invariant to how the keys
+// are split, so the epilogue merges the two partial results exactly:
+//   m = max(m_0, m_1),  l = l_0 2^{m_0 - m} + l_1 2^{m_1 - m},
+//   out = (O_0 2^{m_0 - m} + O_1 2^{m_1 - m}) / l
+// (the sink is counted once, in warpgroup 0's seed).  While one warpgroup
+// waits for its next S, the other works on its own step; with two CTAs per
+// SM, four softmax warps share each SM sub-partition's exp2 unit.  A
+// warpgroup may rescale its
+// O_b without waiting for an MMA: the commit that announced S_h came after
+// the previous PV into O_b (tcgen05 MMAs of one thread execute in order).
 // Tiles outside the causal / window / document range are never visited; only
-// the edge tiles apply an element mask.
+// the edge steps apply an element mask.
 //
-// Warp roles (192 threads, 2 CTAs per SM so one CTA's softmax overlaps the
-// other's MMAs): warps 0-3 softmax + epilogue, warp 4 TMA producer, warp 5
-// TMEM allocator + MMA issuer.  TMEM: S/P in columns [0,128), O in [128,192).
+// Warp roles (320 threads, 2 CTAs per SM): warps 0-7 softmax + epilogue (two
+// warpgroups), warp 8 TMA producer, warp 9 TMEM allocator + MMA issuer.
+// TMEM: S/P buffers in columns [0,64) and [64,128), O_0 in [128,192), O_1 in
+// [192,256).
 #pragma once
 #include "common.cuh"
 
 namespace sa {
 
 constexpr int kFwdStages = 2;
-constexpr int kFwdThreads = 192;
+constexpr int kFwdThreads = 320;
+constexpr int kFwdProducerWarp = 8;
+constexpr int kFwdMmaWarp = 9;
+constexpr int kHalfN = kBlockN / 2;  // keys per softmax step
+constexpr int kHalfBytes = kHalfN * kHeadDim * 2;
 constexpr uint32_t kFwdTmemCols = 256;
 constexpr uint32_t kFwdTmemS = 0;
 constexpr uint32_t kFwdTmemO = 128;
-// The reference max is raised only when a tile's max exceeds it by more than
+// The reference max is raised only when a step's max exceeds it by more than
 // this many powers of two; P <= 2^8 in between, which fp32 and bf16 hold
 // exactly in range.  The result is the same softmax (only rounding differs).
 constexpr float kRescaleLog2 = 8.0f;
@@ -49,9 +67,12 @@ struct FwdCtl {
   uint64_t k_full[kFwdStages];
   uint64_t v_full[kFwdStages];
   uint64_t kv_empty[kFwdStages];
-  uint64_t s_full;
-  uint64_t p_full;
-  uint64_t o_full;
+  uint64_t s_full[2];   // S_h computed into buffer h % 2
+  uint64_t p_full[2];   // P_h written into buffer h % 2 (128 arrivals)
+  uint64_t o_full;      // every MMA done (epilogue may read O_0, O_1)
+  uint64_t merge;       // both warpgroups published their (m, l) (256 arrivals)
+  float m_part[2][kBlockM];
+  float l_part[2][kBlockM];
   uint32_t tmem_base;
   int abort;
 };
@@ -65,7 +86,8 @@ struct FwdTile {
   int t_last;  // last valid token of the tile
   int kv_lo;   // first key any row may see
   int lo_max;  // first key the last row may see (largest over rows)
-  int n_tiles; // key tiles to visit
+  int n_half;  // 64-key steps to visit
+  int n_tiles; // 128-key K/V tiles to load
 };
 
 __device__ __forceinline__ FwdTile fwd_tile(const Geometry& geo) {
@@ -77,12 +99,14 @@ __device__ __forceinline__ FwdTile fwd_tile(const Geometry& geo) {
   w.t_last = min(w.t0 + (1 << geo.P_log2) - 1, geo.T - 1);
   w.kv_lo = first_key(geo, w.t0);
   w.lo_max = first_key(geo, w.t_last);
-  w.n_tiles = (w.t_last - w.kv_lo + kBlockN) / kBlockN;
+  w.n_half = (w.t_last - w.kv_lo + kHalfN) / kHalfN;
+  w.n_tiles = (w.n_half + 1) / 2;
   return w;
 }
 
+// S (64 columns) = Q K^T for the 64 keys whose K rows start at k_addr.
 __device__ __forceinline__ void fwd_issue_qk(uint32_t tmem_s, uint32_t q_addr, uint32_t k_addr) {
-  constexpr uint32_t idesc = make_idesc_bf16(kBlockM, kBlockN, 0, 0);
+  constexpr uint32_t idesc = make_idesc_bf16(kBlockM, kHalfN, 0, 0);
 #pragma unroll
   for (int kk = 0; kk < kHeadDim / 16; ++kk) {
     const uint64_t a = make_sdesc_sw128(q_addr + kk * 32, 16, 1024);
@@ -91,37 +115,46 @@ __device__ __forceinline__ void fwd_issue_qk(uint32_t tmem_s, uint32_t q_addr, u
   }
 }
 
+// O += P V for the 64 keys whose V rows start at v_addr; P (bf16 pairs) in
+// the 32 TMEM columns at tmem_p.
 __device__ __forceinline__ void fwd_issue_pv(uint32_t tmem_o, uint32_t tmem_p, uint32_t v_addr, bool accumulate) {
   constexpr uint32_t idesc = make_idesc_bf16(kBlockM, kHeadDim, 0, 1);
 #pragma unroll
-  for (int kk = 0; kk < kBlockN / 16; ++kk) {
+  for (int kk = 0; kk < kHalfN / 16; ++kk) {
     const uint64_t b = make_sdesc_sw128(v_addr + kk * 2048, kTileBytes, 1024);
     mma_ts(tmem_o, tmem_p + kk * 8, b, idesc, (accumulate || kk > 0) ? 1u : 0u);
   }
 }
 
-// One key tile of one query row: mask (kMask), row max, lazily raised
-// reference max, P = 2^(S*scale*log2e - m) packed to bf16 pairs in s[0..63],
-// and the row sum of P.  s[] holds the row's 128 fp32 logits on entry.
+// One 64-key step of one query row: mask (kMask), row max, lazily raised
+// reference max, P = 2^(S*scale*log2e - m) packed to bf16 pairs in s[0..31],
+// and the row sum of P.  s[] holds the row's 64 fp32 logits on entry.
 struct FwdRowStep {
   bool need;    // the reference max was raised
   float alpha;  // factor applied to the running sum / O (1 when not raised)
-  float m_new;  // reference max after this tile
-  float sum;    // sum of this tile's P
+  float m_new;  // reference max after this step
+  float sum;    // sum of this step's P
 };
 
 template <bool kMask>
 __device__ __forceinline__ FwdRowStep fwd_row_step(uint32_t* s, int c_lo, int c_hi, float sl2, float m_ref) {
-  float x[kBlockN];
+  float x[kHalfN];
 #pragma unroll
-  for (int c = 0; c < kBlockN; ++c) {
+  for (int c = 0; c < kHalfN; ++c) {
     x[c] = __uint_as_float(s[c]);
     if (kMask) x[c] = (c < c_lo || c > c_hi) ? -INFINITY : x[c];
   }
-  float mx = fmax3(x[0], x[1], x[2]);
+  // Row max as four independent chains of 3-input maxima, then combined.
+  float m4[4];
 #pragma unroll
-  for (int c = 3; c < kBlockN - 1; c += 2) mx = fmax3(mx, x[c], x[c + 1]);
-  mx = fmaxf(mx, x[kBlockN - 1]);
+  for (int i = 0; i < 4; ++i) m4[i] = fmax3(x[i], x[i + 4], x[i + 8]);
+#pragma unroll
+  for (int c = 12; c < kHalfN - 4; c += 8) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) m4[i] = fmax3(m4[i], x[c + i], x[c + 4 + i]);
+  }
+  const float mx = fmax3(fmaxf(m4[0], x[kHalfN - 4]), fmax3(m4[1], x[kHalfN - 3], x[kHalfN - 2]),
+                         fmax3(m4[2], m4[3], x[kHalfN - 1]));
   const float mx2 = mx * sl2;
   FwdRowStep r;
   r.need = mx2 > m_ref + kRescaleLog2;
@@ -130,7 +163,7 @@ __device__ __forceinline__ FwdRowStep fwd_row_step(uint32_t* s, int c_lo, int c_
   const float m_use = (r.m_new == -INFINITY) ? 0.f : r.m_new;
   float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-  for (int c = 0; c < kBlockN / 2; ++c) {
+  for (int c = 0; c < kHalfN / 2; ++c) {
     const float e0 = ex2_approx(fmaf(x[2 * c], sl2, -m_use));
     const float e1 = ex2_approx(fmaf(x[2 * c + 1], sl2, -m_use));
     acc[(2 * c) & 3] += e0;
@@ -162,13 +195,16 @@ __global__ void __launch_bounds__(kFwdThreads, 2)
       mbar_init(&ctl->v_full[s], 1);
       mbar_init(&ctl->kv_empty[s], 1);
     }
-    mbar_init(&ctl->s_full, 1);
-    mbar_init(&ctl->p_full, 128);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&ctl->s_full[b], 1);
+      mbar_init(&ctl->p_full[b], kBlockM);
+    }
     mbar_init(&ctl->o_full, 1);
+    mbar_init(&ctl->merge, 2 * kBlockM);
     ctl->abort = 0;
     fence_mbar_init();
   }
-  if (warp == 5) {
+  if (warp == kFwdMmaWarp) {
     tmem_alloc(&ctl->tmem_base, kFwdTmemCols);
     tmem_relinquish();
   }
@@ -177,7 +213,7 @@ __global__ void __launch_bounds__(kFwdThreads, 2)
   tc_fence_after();
   const uint32_t tmem = ctl->tmem_base;
 
-  if (warp == 4) {
+  if (warp == kFwdProducerWarp) {
     // ---------------------------------------------------------- TMA producer
     if (elect_one()) {
       tma_prefetch_desc(&tm_q);
@@ -198,40 +234,50 @@ __global__ void __launch_bounds__(kFwdThreads, 2)
         tma_load_3d(sV + s * kTileBytes, &tm_v, &ctl->v_full[s], 0, w.g, ts);
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == kFwdMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
+    // Order: S_0, S_1, then for every step h: O_{h%2} += P_h V_h, S_{h+2}
+    // into the buffer P_h just left (tcgen05 MMAs of one thread execute in
+    // order, so the PV reads P_h before S_{h+2} overwrites it).
     if (elect_one()) {
       const uint32_t tS = tmem + kFwdTmemS;
       const uint32_t tO = tmem + kFwdTmemO;
       const uint32_t q_addr = smem_u32(sQ);
       bool ok = mbar_wait(&ctl->q_full, 0, abort, &g_device_error, kDevErrTimeoutMma);
-      for (int j = 0; ok && j <= w.n_tiles; ++j) {
-        if (j > 0) {
-          // O += P_{j-1} V_{j-1}
-          const int sp = (j - 1) % kFwdStages;
-          const uint32_t php = ((j - 1) / kFwdStages) & 1;
-          ok = mbar_wait(&ctl->v_full[sp], php, abort, &g_device_error, kDevErrTimeoutMma) &&
-               mbar_wait(&ctl->p_full, (j - 1) & 1, abort, &g_device_error, kDevErrTimeoutMma);
-          if (!ok) break;
-          tc_fence_after();
-          fwd_issue_pv(tO, tS, smem_u32(sV + sp * kTileBytes), j > 1);
-          tc_commit(&ctl->kv_empty[sp]);
-        }
-        if (j == w.n_tiles) break;
-        // S = Q K_j^T (overwrites P_{j-1}: the PV above was issued first and
-        // tcgen05 MMAs from one thread execute in order).
-        const int s = j % kFwdStages;
-        ok = mbar_wait(&ctl->k_full[s], (j / kFwdStages) & 1, abort, &g_device_error, kDevErrTimeoutMma);
+      for (int h = 0; ok && h < min(2, w.n_half); ++h) {
+        ok = mbar_wait(&ctl->k_full[0], 0, abort, &g_device_error, kDevErrTimeoutMma);
         if (!ok) break;
         tc_fence_after();
-        fwd_issue_qk(tS, q_addr, smem_u32(sK + s * kTileBytes));
-        tc_commit(&ctl->s_full);
+        fwd_issue_qk(tS + h * kHalfN, q_addr, smem_u32(sK) + h * kHalfBytes);
+        tc_commit(&ctl->s_full[h]);
+      }
+      for (int h = 0; ok && h < w.n_half; ++h) {
+        const int b = h & 1;
+        const int j = h >> 1;
+        const int s = j % kFwdStages;
+        ok = mbar_wait(&ctl->v_full[s], (j / kFwdStages) & 1, abort, &g_device_error, kDevErrTimeoutMma) &&
+             mbar_wait(&ctl->p_full[b], (h >> 1) & 1, abort, &g_device_error, kDevErrTimeoutMma);
+        if (!ok) break;
+        tc_fence_after();
+        fwd_issue_pv(tO + b * kHeadDim, tS + b * kHalfN, smem_u32(sV + s * kTileBytes) + b * kHalfBytes, h >= 2);
+        if (b == 1 || h == w.n_half - 1) tc_commit(&ctl->kv_empty[s]);
+        const int h2 = h + 2;
+        if (h2 < w.n_half) {
+          const int j2 = h2 >> 1;
+          const int s2 = j2 % kFwdStages;
+          ok = mbar_wait(&ctl->k_full[s2], (j2 / kFwdStages) & 1, abort, &g_device_error, kDevErrTimeoutMma);
+          if (!ok) break;
+          tc_fence_after();
+          fwd_issue_qk(tS + b * kHalfN, q_addr, smem_u32(sK + s2 * kTileBytes) + b * kHalfBytes);
+          tc_commit(&ctl->s_full[b]);
+        }
       }
       if (ok) tc_commit(&ctl->o_full);
     }
   } else {
-    // ------------------------------------------------------ softmax (1 row)
-    const int r = threadIdx.x;
+    // ------------------------------------------- softmax (1 row per thread)
+    const int wg = warp >> 2;  // steps h with h % 2 == wg
+    const int r = threadIdx.x & (kBlockM - 1);
     const int G = 1 << geo.G_log2;
     const int t = w.t0 + (r >> geo.G_log2);
     const int h = (w.g << geo.G_log2) + (r & (G - 1));
@@ -242,79 +288,101 @@ __global__ void __launch_bounds__(kFwdThreads, 2)
       hi_r = t;
     }
     const float sink = __ldg(p.sinks + h);
-    float m_ref = sink * kLog2e;                 // -inf when the sink is off
-    float l = (sink == -INFINITY) ? 0.f : 1.f;   // e^{s - m} with m = s
-    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-    const uint32_t tS = tmem + lane_base + kFwdTmemS;
-    const uint32_t tO = tmem + lane_base + kFwdTmemO;
+    // Both warpgroups take the sink logit as their first reference max; only
+    // warpgroup 0 counts the sink's own e^{s-m} = 1 in its sum.
+    float m_ref = sink * kLog2e;  // -inf when the sink is off
+    float l = (wg == 0 && sink != -INFINITY) ? 1.f : 0.f;
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + lane_base + kFwdTmemS + wg * kHalfN;
+    const uint32_t tO = tmem + lane_base + kFwdTmemO + wg * kHeadDim;
     const float sl2 = p.scale_log2;
     bool ok = true;
 
-    for (int j = 0; j < w.n_tiles; ++j) {
-      ok = mbar_wait(&ctl->s_full, j & 1, abort, &g_device_error, kDevErrTimeoutSoftmax);
+    for (int hs = wg, i = 0; hs < w.n_half; hs += 2, ++i) {
+      ok = mbar_wait(&ctl->s_full[wg], i & 1, abort, &g_device_error, kDevErrTimeoutSoftmax);
       if (!ok) break;
       tc_fence_after();
-      uint32_t sr[kBlockN];
+      uint32_t sr[kHalfN];
       tmem_ld64(tS, sr);
-      tmem_ld64(tS + 64, sr + 64);
-      const int ts = w.kv_lo + j * kBlockN;
-      // CTA-uniform: does any row of this tile see a masked key?  Resolved
-      // once per tile, not per element.
+      const int ks = w.kv_lo + hs * kHalfN;
+      // CTA-uniform: does any row of this step see a masked key?  Resolved
+      // once per step, not per element.
       FwdRowStep st;
-      if (ts + kBlockN - 1 > w.t0 || ts < w.lo_max)
-        st = fwd_row_step<true>(sr, lo_r - ts, hi_r - ts, sl2, m_ref);
+      if (ks + kHalfN - 1 > w.t0 || ks < w.lo_max)
+        st = fwd_row_step<true>(sr, lo_r - ks, hi_r - ks, sl2, m_ref);
       else
         st = fwd_row_step<false>(sr, 0, 0, sl2, m_ref);
-      const bool need = st.need;
-      const float alpha = st.alpha;
-      const float m_new = st.m_new;
-      l = l * alpha + st.sum;
-      uint32_t* pk = sr;  // fwd_row_step packed P (bf16 pairs) into sr[0..63]
+      l = l * st.alpha + st.sum;
       __syncwarp();
-      tmem_st32(tS, pk);
-      tmem_st32(tS + 32, pk + 32);
-      // Rescale the running O (TMEM) when a row of this warp raised its
-      // reference max.  O_{j-1} is complete: the S_j commit came after it.
-      if (j > 0 && __any_sync(0xffffffffu, need)) {
+      tmem_st32(tS, sr);  // fwd_row_step packed P (bf16 pairs) into sr[0..31]
+      // Rescale this warpgroup's O when a row of the warp raised its
+      // reference max.  Its previous PV is complete: it was issued before
+      // the S MMA whose commit was just observed.
+      if (i > 0 && __any_sync(0xffffffffu, st.need)) {
         uint32_t o[kHeadDim];
         tmem_ld64(tO, o);
 #pragma unroll
-        for (int i = 0; i < kHeadDim; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+        for (int c = 0; c < kHeadDim; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * st.alpha);
         tmem_st32(tO, o);
         tmem_st32(tO + 32, o + 32);
       }
-      m_ref = m_new;
+      m_ref = st.m_new;
       tc_fence_before();
-      mbar_arrive(&ctl->p_full);
+      mbar_arrive(&ctl->p_full[wg]);
     }
 
-    // ----------------------------------------------------------- epilogue
+    // ------------------------------------------------ merge and epilogue
+    // Each warpgroup publishes its (m, l); then warpgroup b writes output
+    // columns [32 b, 32 b + 32) of its rows from both accumulators.
     if (ok) ok = mbar_wait(&ctl->o_full, 0, abort, &g_device_error, kDevErrTimeoutEpilogue);
+    ctl->m_part[wg][r] = m_ref;
+    ctl->l_part[wg][r] = l;
+    uint32_t merge_phase = 0;
+    mbar_arrive(&ctl->merge);
+    if (ok) ok = mbar_wait(&ctl->merge, merge_phase, abort, &g_device_error, kDevErrTimeoutEpilogue);
     if (ok) {
       tc_fence_after();
-      uint32_t o[kHeadDim];
+      const bool has1 = w.n_half >= 2;  // warpgroup 1 saw at least one step
+      const float m0 = ctl->m_part[0][r], l0 = ctl->l_part[0][r];
+      const float m1 = has1 ? ctl->m_part[1][r] : -INFINITY;
+      const float l1 = has1 ? ctl->l_part[1][r] : 0.f;
+      const float m = fmaxf(m0, m1);
+      const float f0 = (m == -INFINITY) ? 0.f : ex2_approx(m0 - m);
+      const float f1 = (m == -INFINITY || !has1) ? 0.f : ex2_approx(m1 - m);
+      const float lt = l0 * f0 + l1 * f1;
+      const uint32_t tO0 = tmem + lane_base + kFwdTmemO + wg * 32;
+      uint32_t o0[32], o1[32];
       __syncwarp();
-      tmem_ld64(tO, o);
+      tmem_ld32(tO0, o0);
+      if (has1) tmem_ld32(tO0 + kHeadDim, o1);
       if (valid) {
-        const float inv_l = l > 0.f ? 1.f / l : 0.f;
-        uint4* dst = reinterpret_cast<uint4*>(p.out + (static_cast<size_t>(t) * geo.Hq + h) * kHeadDim);
+        const float inv_l = lt > 0.f ? 1.f / lt : 0.f;
+        const float g0 = f0 * inv_l, g1 = f1 * inv_l;
+        uint4* dst = reinterpret_cast<uint4*>(p.out + (static_cast<size_t>(t) * geo.Hq + h) * kHeadDim + wg * 32);
 #pragma unroll
-        for (int i = 0; i < kHeadDim / 8; ++i) {
+        for (int c8 = 0; c8 < 4; ++c8) {
+          float y[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const int c = 8 * c8 + u;
+            y[u] = __uint_as_float(o0[c]) * g0;
+            if (has1) y[u] = fmaf(__uint_as_float(o1[c]), g1, y[u]);
+          }
           uint4 v;
-          v.x = pack_bf16x2(__uint_as_float(o[8 * i + 0]) * inv_l, __uint_as_float(o[8 * i + 1]) * inv_l);
-          v.y = pack_bf16x2(__uint_as_float(o[8 * i + 2]) * inv_l, __uint_as_float(o[8 * i + 3]) * inv_l);
-          v.z = pack_bf16x2(__uint_as_float(o[8 * i + 4]) * inv_l, __uint_as_float(o[8 * i + 5]) * inv_l);
-          v.w = pack_bf16x2(__uint_as_float(o[8 * i + 6]) * inv_l, __uint_as_float(o[8 * i + 7]) * inv_l);
-          dst[i] = v;
+          v.x = pack_bf16x2(y[0], y[1]);
+          v.y = pack_bf16x2(y[2], y[3]);
+          v.z = pack_bf16x2(y[4], y[5]);
+          v.w = pack_bf16x2(y[6], y[7]);
+          dst[c8] = v;
         }
-        p.lse[static_cast<size_t>(h) * geo.T + t] = l > 0.f ? (m_ref + __log2f(l)) * kLn2 : -INFINITY;
+        if (wg == 0) p.lse[static_cast<size_t>(h) * geo.T + t] = lt > 0.f ? (m + __log2f(lt)) * kLn2 : -INFINITY;
       }
     }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == kFwdMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, kFwdTmemCols);
   }
