@@ -151,6 +151,66 @@ sink_attn_status sink_attn_bwd_noalloc(const sink_attn_dims* dims,
                                        void* dq, void* dk, void* dv, float* dsinks,
                                        void* stream);
 
+/* ------------------------------------------------------------------ decode
+ * Decode forward over a key/value cache: a few new tokens per sequence are
+ * appended to the cache and their queries attend to everything the cache
+ * holds for that sequence, with the same sink, window and causal rules as
+ * sink_attn_fwd().  This is the incremental form of the forward the pages use
+ * for generation with the alternating sliding-window / full layers
+ * ("Tricks from OpenAI gpt-oss you can use with transformers", list item
+ * "Dynamic Sliding Window Layer & Cache"); the pages do not describe the
+ * cache itself, so its layout is this library's own:
+ *
+ *   - Sequence b owns cache_capacity (C) slots of k_cache / v_cache, each
+ *     slot [Hkv][D] bf16: k_cache, v_cache are [batch][C][Hkv][D].  The token
+ *     at position p lives in slot p mod C.  With C >= every sequence length
+ *     this is a plain linear cache; a sliding-window layer may keep a ring of
+ *     C >= window + new_tokens - 1 slots, which holds every key a new query
+ *     can see.  A ring smaller than that loses keys: the kernel then records
+ *     device error 0x201 (see sink_attn_device_error) and its output is not
+ *     defined.
+ *   - cache_seqlens [batch] (int32, device) = L0_b, the tokens of sequence b
+ *     in the cache before this call.  The call writes the new tokens at
+ *     positions L0_b .. L0_b + new_tokens - 1 (slots mod C) and does not
+ *     modify cache_seqlens; the caller advances it by new_tokens.
+ *   - New query t of sequence b has position i = L0_b + t and sees key
+ *     position j iff j <= i and (window <= 0 or i - j < window).
+ */
+typedef struct {
+    int batch;          /* sequences */
+    int new_tokens;     /* Lq >= 1: new tokens per sequence (1 for one-token decode) */
+    int cache_capacity; /* C: slots per sequence */
+    int max_seqlen;     /* upper bound on L0_b + new_tokens over b (sizes the split grid) */
+    int num_q_heads;    /* Hq */
+    int num_kv_heads;   /* Hkv */
+    int head_dim;       /* D (64) */
+} sink_attn_decode_dims;
+
+/* Bytes of device workspace sink_attn_decode() needs (per-split partial
+ * results); 0 when the sizes are invalid.  Depends on `window`. */
+size_t sink_attn_decode_workspace_size(const sink_attn_decode_dims* dims, int window);
+
+/* Decode.  q [batch][new_tokens][Hq][D] bf16, k_new / v_new
+ * [batch][new_tokens][Hkv][D] bf16 (appended to the cache by this call),
+ * k_cache / v_cache as above (read and written), cache_seqlens as above,
+ * sinks [Hq] fp32.  Writes out [batch][new_tokens][Hq][D] bf16 and
+ * lse [Hq][batch * new_tokens] fp32 (natural log, sink included).
+ * Supported: D = 64, G = Hq / Hkv a power of two with G * new_tokens <= 64.
+ * `workspace`: caller-owned device memory of at least
+ * sink_attn_decode_workspace_size(dims, window) bytes, 256-byte aligned.
+ * batch = 0 is a no-op.  Launches three kernels (append, attend, combine)
+ * on `stream`. */
+sink_attn_status sink_attn_decode(const sink_attn_decode_dims* dims,
+                                  const void* q, const void* k_new, const void* v_new,
+                                  void* k_cache, void* v_cache, const int* cache_seqlens,
+                                  const float* sinks, int window, float scale,
+                                  void* out, float* lse,
+                                  void* workspace, size_t workspace_bytes,
+                                  void* stream);
+
+/* Number of kernels one sink_attn_decode call launches (0 when batch = 0). */
+int sink_attn_decode_launches(const sink_attn_decode_dims* dims);
+
 /* Human-readable name of a status code (static string, never NULL). */
 const char* sink_attn_status_string(sink_attn_status s);
 

@@ -1,0 +1,522 @@
+// Decode forward: a few new query tokens per sequence attend to that
+// sequence's key/value cache (sink, sliding window and causal mask as in the
+// forward).  Three kernels per call: append the new keys/values to the cache,
+// attend (split over the cache), combine the splits.
+//
+// Cache layout.  Sequence b owns `C` slots of k_cache / v_cache, each slot
+// [Hkv][D]; the token at position p lives in slot p mod C.  A cache with
+// C >= the sequence length is a plain linear cache; a sliding-window layer
+// can keep a ring of C >= window + new_tokens - 1 slots.  Before a call the
+// cache holds positions [0, L0) (the last C of them), L0 = cache_seqlens[b];
+// the call writes the Lq new tokens at positions L0 .. L0+Lq-1 and their
+// queries attend with the same masks as the forward: key position j is
+// allowed for query position i iff j <= i and (window <= 0 or i - j < window).
+//
+// Attention kernel (one CTA = sequence b, key/value head g, one split of
+// the cache slots).  With only G x Lq (<= 64) query rows per head group, the
+// MMA roles are swapped so the keys fill the 128-row M dimension:
+//   S^T = K Q^T           M = 128 keys of a slot tile, N = 64 query rows
+//                         (G x Lq real, the rest zero), K = D
+//   softmax over keys     one thread per key (its TMEM lane); the per-row
+//                         reference max is shared by all threads (seeded
+//                         with the sink logit, raised lazily: only when some
+//                         key exceeds it by more than 2^8, found by a vote)
+//   O^T += [V | 1]^T P^T  M = 128: rows 0..63 are the head dims (A = V read
+//                         MN-major), rows 64..127 multiply P^T by a tile of
+//                         ones and so accumulate the row sums l for free;
+//                         B = P^T [keys][rows] written to shared memory
+// Softmax is invariant to the order of the keys, so slots are visited in
+// slot order; each key's position (and so its mask) follows from the slot.
+// Each split writes (O, l, m) partials; the combine kernel merges them and
+// adds the sink's e^{s-m} once.
+#pragma once
+#include "common.cuh"
+
+namespace sa {
+
+constexpr int kDecThreads = 192;  // warps 0-3 softmax (one key per thread), 4 TMA producer, 5 MMA
+constexpr int kDecProducerWarp = 4;
+constexpr int kDecMmaWarp = 5;
+constexpr int kDecRows = 64;      // MMA N: query rows per CTA (G x Lq <= 64)
+constexpr int kDecTile = 128;     // slots per key tile (MMA M)
+constexpr int kDecStages = 2;
+constexpr int kDecQBytes = kDecRows * kHeadDim * 2;    // Q tile, [64][64] bf16
+constexpr int kDecKvBytes = kDecTile * kHeadDim * 2;   // one K or V tile, [128][64] bf16
+constexpr int kDecPBytes = kDecTile * kDecRows * 2;    // P^T tile, [128 keys][64 rows] bf16
+constexpr uint32_t kDecTmemCols = 256;  // S^T buffers [0,64), [64,128); O^T [128,192)
+constexpr uint32_t kDecTmemS = 0;
+constexpr uint32_t kDecTmemO = 128;
+constexpr float kDecRescaleLog2 = 8.0f;
+
+struct DecParams {
+  int batch, Lq, C, Hq, Hkv, G, R;  // R = G * Lq query rows per (sequence, kv head)
+  int G_log2;                       // G is a power of two
+  int window;                       // <= 0: full causal
+  int n_split;                      // CTAs per (sequence, kv head)
+  float scale_log2;                 // scale * log2(e)
+  const int* seqlens;               // [batch] tokens in the cache before this call
+  const float* sinks;               // [Hq]
+  float* o_part;                    // [batch][Hkv][n_split][64 rows][64] unnormalised O
+  float* m_part;                    // [batch][Hkv][n_split][64 rows] reference max (log2 units)
+  float* l_part;                    // [batch][Hkv][n_split][64 rows] sum of P
+};
+
+struct DecCtl {
+  uint64_t q_full;
+  uint64_t k_full[kDecStages];
+  uint64_t k_empty[kDecStages];
+  uint64_t v_full[kDecStages];
+  uint64_t v_empty[kDecStages];
+  uint64_t s_full[2];   // S^T of tile i in TMEM buffer i % 2
+  uint64_t s_free[2];   // the softmax has loaded that S^T (128 arrivals)
+  uint64_t p_full;      // P^T of tile i written (128 arrivals)
+  uint64_t pv_done;     // O^T += ... of tile i complete
+  uint64_t o_full;      // every MMA done
+  uint64_t sync;        // the 128 softmax threads
+  float m_ref[kDecRows];    // reference max per query row (log2 units)
+  float alpha[kDecRows];    // rescale factor of the current tile per row
+  float wmax[4][kDecRows];  // per-warp tile maxima (rare path)
+  int vote[2][4];           // per-warp "a key exceeds the reference" flags, by tile parity
+  uint32_t tmem_base;
+  int abort;
+};
+
+constexpr size_t kDecSmemBytes = 1024 /*alignment slack*/ + kDecQBytes + 2 * kDecStages * kDecKvBytes +
+                                 kDecKvBytes /*ones*/ + kDecPBytes + sizeof(DecCtl);
+
+// Slot range of one CTA: [z0, z0 + 128 n) in 128-slot tiles.
+struct DecWork {
+  int b, g, split;
+  int L0, L;     // cache length before / after this call
+  int z0;        // first slot of the first tile
+  int n;         // tiles to visit (may be 0)
+  bool bad;      // a needed key is no longer in the cache
+};
+
+__device__ __forceinline__ DecWork dec_work(const DecParams& p) {
+  DecWork w;
+  const int bg = blockIdx.x / p.n_split;
+  w.split = blockIdx.x % p.n_split;
+  w.b = bg / p.Hkv;
+  w.g = bg % p.Hkv;
+  w.L0 = __ldg(p.seqlens + w.b);
+  w.L = w.L0 + p.Lq;
+  if (w.L0 < 0) {  // invalid length: visit nothing, report it
+    w.z0 = 0;
+    w.n = 0;
+    w.bad = true;
+    return w;
+  }
+  // Oldest position any new query may see.
+  const int pmin = p.window > 0 ? max(0, w.L0 - p.window + 1) : 0;
+  int zlo, zhi;  // slots to scan
+  if (w.L <= p.C) {
+    zlo = pmin;  // no wrap: slot == position
+    zhi = w.L;
+    w.bad = false;
+  } else {
+    zlo = 0;     // wrapped ring: every slot holds one of the last C positions
+    zhi = p.C;
+    w.bad = pmin < w.L - p.C;
+  }
+  const int t_first = zlo / kDecTile;
+  const int t_count = (zhi + kDecTile - 1) / kDecTile - t_first;
+  const int per = (t_count + p.n_split - 1) / p.n_split;
+  const int t_begin = min(t_count, w.split * per);
+  w.n = min(t_count, t_begin + per) - t_begin;
+  w.z0 = (t_first + t_begin) * kDecTile;
+  return w;
+}
+
+// Position of the token in slot z (negative: the slot holds no token yet).
+__device__ __forceinline__ int dec_slot_pos(int z, int L, int C) {
+  int d = (L - 1 - z) % C;
+  if (d < 0) d += C;
+  return L - 1 - d;
+}
+
+// S^T (64 columns) = K Q^T: A = the K tile (128 slots, K-major), B = Q
+// (64 rows, K-major).
+__device__ __forceinline__ void dec_issue_qk(uint32_t tmem_s, uint32_t k_addr, uint32_t q_addr) {
+  constexpr uint32_t idesc = make_idesc_bf16(kDecTile, kDecRows, 0, 0);
+#pragma unroll
+  for (int kk = 0; kk < kHeadDim / 16; ++kk) {
+    const uint64_t a = make_sdesc_sw128(k_addr + kk * 32, 16, 1024);
+    const uint64_t b = make_sdesc_sw128(q_addr + kk * 32, 16, 1024);
+    mma_ss(tmem_s, a, b, idesc, kk > 0 ? 1u : 0u);
+  }
+}
+
+// O^T (+)= [V | 1]^T P^T over the 128 slots of a tile: A (M = 128) is read
+// MN-major from the V tile (M rows 0..63) and the ones tile (M rows 64..127,
+// reached through the descriptor's leading-byte offset); B = P^T [slots][64
+// rows], MN-major.
+__device__ __forceinline__ void dec_issue_pv(uint32_t tmem_o, uint32_t v_addr, uint32_t ones_addr, uint32_t p_addr,
+                                             bool accumulate) {
+  constexpr uint32_t idesc = make_idesc_bf16(kDecTile, kDecRows, 1, 1);
+  const uint32_t lbo = ones_addr - v_addr;
+#pragma unroll
+  for (int kk = 0; kk < kDecTile / 16; ++kk) {
+    const uint64_t a = make_sdesc_sw128(v_addr + kk * 2048, lbo, 1024);
+    const uint64_t b = make_sdesc_sw128(p_addr + kk * 2048, kDecPBytes, 1024);
+    mma_ss(tmem_o, a, b, idesc, (accumulate || kk > 0) ? 1u : 0u);
+  }
+}
+
+__device__ __forceinline__ bool dec_group_sync(DecCtl* ctl, uint32_t& phase, volatile int* abort) {
+  mbar_arrive(&ctl->sync);
+  const bool ok = mbar_wait(&ctl->sync, phase, abort, &g_device_error, kDevErrTimeoutDecode);
+  phase ^= 1u;
+  return ok;
+}
+
+// Loads / stores kN (16, 32 or 64) consecutive TMEM columns of this warp's lanes.
+template <int kN>
+__device__ __forceinline__ void dec_tmem_ld(uint32_t taddr, uint32_t* r) {
+  if constexpr (kN == 16) tmem_ld16(taddr, r);
+  else if constexpr (kN == 32) tmem_ld32(taddr, r);
+  else tmem_ld64(taddr, r);
+}
+template <int kN>
+__device__ __forceinline__ void dec_tmem_st(uint32_t taddr, const uint32_t* r) {
+  if constexpr (kN == 16) {
+    tmem_st16(taddr, r);
+  } else {
+#pragma unroll
+    for (int c = 0; c < kN / 32; ++c) tmem_st32(taddr + 32 * c, r + 32 * c);
+  }
+}
+
+// kR: query rows handled in registers (16, 32 or 64; >= G * Lq).
+template <int kR>
+__global__ void __launch_bounds__(kDecThreads, 2)
+    sink_attn_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                            const __grid_constant__ CUtensorMap tm_v, const DecParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint8_t* sK = smem;                                   // stages of K tiles
+  uint8_t* sV = sK + kDecStages * kDecKvBytes;          // stages of V tiles
+  uint8_t* sOnes = sV + kDecStages * kDecKvBytes;       // [128][64] bf16 ones
+  uint8_t* sP = sOnes + kDecKvBytes;                    // P^T
+  uint8_t* sQ = sP + kDecPBytes;                        // Q rows (8 KB, 1024-aligned)
+  DecCtl* ctl = reinterpret_cast<DecCtl*>(sQ + kDecQBytes);
+  volatile int* abort = &ctl->abort;
+  const int warp = threadIdx.x >> 5;
+  const DecWork w = dec_work(p);
+
+  if (threadIdx.x == 0) {
+    mbar_init(&ctl->q_full, 1);
+    for (int s = 0; s < kDecStages; ++s) {
+      mbar_init(&ctl->k_full[s], 1);
+      mbar_init(&ctl->k_empty[s], 1);
+      mbar_init(&ctl->v_full[s], 1);
+      mbar_init(&ctl->v_empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&ctl->s_full[b], 1);
+      mbar_init(&ctl->s_free[b], kDecTile);
+    }
+    mbar_init(&ctl->p_full, kDecTile);
+    mbar_init(&ctl->pv_done, 1);
+    mbar_init(&ctl->o_full, 1);
+    mbar_init(&ctl->sync, kDecTile);
+    ctl->abort = 0;
+    if (w.bad) atomicCAS(&g_device_error, 0, static_cast<int>(kDevErrDecodeCacheTooSmall));
+    fence_mbar_init();
+  }
+  if (threadIdx.x < kDecRows) {
+    float m0 = -INFINITY;
+    if (threadIdx.x < p.R) m0 = __ldg(p.sinks + w.g * p.G + (threadIdx.x & (p.G - 1))) * kLog2e;
+    ctl->m_ref[threadIdx.x] = m0;
+    ctl->alpha[threadIdx.x] = 1.f;
+  }
+  // Constant operands written by the threads: the ones tile, zeroed P^T and
+  // zeroed Q padding rows (the TMA fills rows [0, R)).
+  {
+    const uint4 ones = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
+    const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
+    for (int i = threadIdx.x; i < kDecKvBytes / 16; i += kDecThreads) {
+      reinterpret_cast<uint4*>(sOnes)[i] = ones;
+      reinterpret_cast<uint4*>(sP)[i] = zero;
+    }
+    for (int i = p.R * 8 + threadIdx.x; i < kDecQBytes / 16; i += kDecThreads) reinterpret_cast<uint4*>(sQ)[i] = zero;
+    fence_proxy_async_smem();
+  }
+  if (warp == kDecMmaWarp) {
+    tmem_alloc(&ctl->tmem_base, kDecTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ctl->tmem_base;
+
+  if (warp == kDecProducerWarp) {
+    // ---------------------------------------------------------- TMA producer
+    if (w.n > 0 && elect_one()) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      mbar_arrive_expect_tx(&ctl->q_full, p.R * kHeadDim * 2);
+      tma_load_3d(sQ, &tm_q, &ctl->q_full, 0, w.g * p.G, w.b * p.Lq);
+      const int row0 = w.b * p.C + w.z0;
+      for (int i = 0; i < w.n; ++i) {
+        const int s = i % kDecStages;
+        const uint32_t par = ((i / kDecStages) - 1) & 1;
+        if (i >= kDecStages && !mbar_wait(&ctl->k_empty[s], par, abort, &g_device_error, kDevErrTimeoutProducer))
+          break;
+        mbar_arrive_expect_tx(&ctl->k_full[s], kDecKvBytes);
+        tma_load_3d(sK + s * kDecKvBytes, &tm_k, &ctl->k_full[s], 0, w.g, row0 + i * kDecTile);
+        if (i >= kDecStages && !mbar_wait(&ctl->v_empty[s], par, abort, &g_device_error, kDevErrTimeoutProducer))
+          break;
+        mbar_arrive_expect_tx(&ctl->v_full[s], kDecKvBytes);
+        tma_load_3d(sV + s * kDecKvBytes, &tm_v, &ctl->v_full[s], 0, w.g, row0 + i * kDecTile);
+      }
+    }
+  } else if (warp == kDecMmaWarp) {
+    // ------------------------------------------------------------ MMA issuer
+    // S^T_i, then O^T += ... for tile i - 1 (its P^T is written while S^T_i
+    // is being computed).
+    if (w.n > 0 && elect_one()) {
+      const uint32_t tS = tmem + kDecTmemS;
+      const uint32_t tO = tmem + kDecTmemO;
+      const uint32_t q_addr = smem_u32(sQ);
+      const uint32_t ones_addr = smem_u32(sOnes);
+      const uint32_t p_addr = smem_u32(sP);
+      bool ok = mbar_wait(&ctl->q_full, 0, abort, &g_device_error, kDevErrTimeoutMma);
+      for (int i = 0; ok && i <= w.n; ++i) {
+        if (i < w.n) {
+          const int b = i & 1;
+          const int s = i % kDecStages;
+          ok = (i < 2 || mbar_wait(&ctl->s_free[b], ((i >> 1) - 1) & 1, abort, &g_device_error, kDevErrTimeoutMma)) &&
+               mbar_wait(&ctl->k_full[s], (i / kDecStages) & 1, abort, &g_device_error, kDevErrTimeoutMma);
+          if (!ok) break;
+          tc_fence_after();
+          dec_issue_qk(tS + b * kDecRows, smem_u32(sK + s * kDecKvBytes), q_addr);
+          tc_commit(&ctl->s_full[b]);
+          tc_commit(&ctl->k_empty[s]);
+        }
+        if (i >= 1) {
+          const int j = i - 1;
+          const int s = j % kDecStages;
+          ok = mbar_wait(&ctl->p_full, j & 1, abort, &g_device_error, kDevErrTimeoutMma) &&
+               mbar_wait(&ctl->v_full[s], (j / kDecStages) & 1, abort, &g_device_error, kDevErrTimeoutMma);
+          if (!ok) break;
+          tc_fence_after();
+          dec_issue_pv(tO, smem_u32(sV + s * kDecKvBytes), ones_addr, p_addr, j > 0);
+          tc_commit(&ctl->pv_done);
+          tc_commit(&ctl->v_empty[s]);
+        }
+      }
+      if (ok) tc_commit(&ctl->o_full);
+    }
+  } else {
+    // ---------------------------------------- softmax (1 key per thread)
+    const int kl = threadIdx.x;  // slot within the tile == TMEM lane
+    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    const float sl2 = p.scale_log2;
+    uint32_t sync_phase = 0;
+    bool ok = true;
+    for (int i = 0; i < w.n; ++i) {
+      const int b = i & 1;
+      ok = mbar_wait(&ctl->s_full[b], (i >> 1) & 1, abort, &g_device_error, kDevErrTimeoutDecode);
+      if (!ok) break;
+      tc_fence_after();
+      float x[kR];
+      {
+        uint32_t raw[kR];
+        dec_tmem_ld<kR>(tmem + lane_base + kDecTmemS + b * kDecRows, raw);
+#pragma unroll
+        for (int n = 0; n < kR; ++n) x[n] = __uint_as_float(raw[n]);
+      }
+      tc_fence_before();
+      mbar_arrive(&ctl->s_free[b]);
+      // Mask: slot -> position -> allowed for each query row.
+      const int z = w.z0 + i * kDecTile + kl;
+      const int pos = z < p.C ? dec_slot_pos(z, w.L, p.C) : -1;
+      bool viol = false;
+#pragma unroll
+      for (int n = 0; n < kR; ++n) {
+        const int qi = w.L0 + (n >> p.G_log2);  // query position of row n
+        const bool allowed = n < p.R && pos >= 0 && pos <= qi && (p.window <= 0 || qi - pos < p.window);
+        x[n] = allowed ? x[n] * sl2 : -INFINITY;
+        viol |= x[n] > ctl->m_ref[n] + kDecRescaleLog2;
+      }
+      // Raise the shared reference max only when some key exceeds it by
+      // more than 2^8 (decided by a vote of all 128 keys).
+      const unsigned any_w = __ballot_sync(0xffffffffu, viol);
+      if ((kl & 31) == 0) ctl->vote[b][warp] = any_w != 0u;
+      ok = dec_group_sync(ctl, sync_phase, abort);
+      if (!ok) break;
+      const bool raise = ctl->vote[b][0] | ctl->vote[b][1] | ctl->vote[b][2] | ctl->vote[b][3];
+      if (raise) {
+#pragma unroll
+        for (int n = 0; n < kR; ++n) {
+          if (n < p.R) {
+            float v = x[n];
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+            if ((kl & 31) == 0) ctl->wmax[warp][n] = v;
+          }
+        }
+        ok = dec_group_sync(ctl, sync_phase, abort);
+        if (!ok) break;
+        if (kl < p.R) {
+          const float tmax = fmaxf(fmaxf(ctl->wmax[0][kl], ctl->wmax[1][kl]), fmaxf(ctl->wmax[2][kl], ctl->wmax[3][kl]));
+          const float mr = ctl->m_ref[kl];
+          const bool up = tmax > mr + kDecRescaleLog2;
+          ctl->alpha[kl] = up ? ex2_approx(mr - tmax) : 1.f;
+          if (up) ctl->m_ref[kl] = tmax;
+        }
+        ok = dec_group_sync(ctl, sync_phase, abort);
+        if (!ok) break;
+      }
+      // P^T row of this key, packed to bf16 pairs (rows 2c, 2c+1).
+      uint32_t pk[kR / 2];
+#pragma unroll
+      for (int c = 0; c < kR / 2; ++c) {
+        const float m0 = ctl->m_ref[2 * c], m1 = ctl->m_ref[2 * c + 1];
+        const float e0 = ex2_approx(x[2 * c] - (m0 == -INFINITY ? 0.f : m0));
+        const float e1 = ex2_approx(x[2 * c + 1] - (m1 == -INFINITY ? 0.f : m1));
+        pk[c] = pack_bf16x2(e0, e1);
+      }
+      // The previous PV read P^T and wrote O^T: wait for it before both.
+      if (i > 0) {
+        ok = mbar_wait(&ctl->pv_done, (i - 1) & 1, abort, &g_device_error, kDevErrTimeoutDecode);
+        if (!ok) break;
+        if (raise) {
+          // O^T[lane][n] *= alpha[n]: head dims in lanes 0..63, row sums in
+          // lanes 64..127, query rows in columns.
+          tc_fence_after();
+          uint32_t o[kR];
+          dec_tmem_ld<kR>(tmem + lane_base + kDecTmemO, o);
+#pragma unroll
+          for (int n = 0; n < kR; ++n) o[n] = __float_as_uint(__uint_as_float(o[n]) * ctl->alpha[n]);
+          dec_tmem_st<kR>(tmem + lane_base + kDecTmemO, o);
+        }
+      }
+      // A slot that holds no token (never written, or past this sequence's
+      // C slots) may hold any bits, NaN included, and its V row is still
+      // multiplied by P = 0: zero that row of the staged V tile.
+      if (pos < 0) {
+        const int sv = i % kDecStages;
+        ok = mbar_wait(&ctl->v_full[sv], (i / kDecStages) & 1, abort, &g_device_error, kDevErrTimeoutDecode);
+        if (!ok) break;
+        uint4* vrow = reinterpret_cast<uint4*>(sV + sv * kDecKvBytes + (kl >> 3) * 1024 + (kl & 7) * 128);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) vrow[c] = make_uint4(0u, 0u, 0u, 0u);
+      }
+      // P^T [slot kl][rows]: 128 B per slot, 16-byte chunk c (rows 8c..8c+7)
+      // at chunk position c ^ (kl % 8).
+      uint8_t* line = sP + (kl >> 3) * 1024 + (kl & 7) * 128;
+#pragma unroll
+      for (int c = 0; c < kR / 8; ++c) {
+        if (c * 8 < p.R)
+          *reinterpret_cast<uint4*>(line + ((c ^ (kl & 7)) << 4)) =
+              make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(&ctl->p_full);
+    }
+
+    // ------------------------------------------------------------ partials
+    const size_t cta = static_cast<size_t>(blockIdx.x);
+    bool have = ok && w.n > 0;
+    if (have) have = mbar_wait(&ctl->o_full, 0, abort, &g_device_error, kDevErrTimeoutEpilogue);
+    if (have) tc_fence_after();
+    if (warp < 3) {
+      uint32_t o[kR];
+      if (have) {
+        __syncwarp();
+        dec_tmem_ld<kR>(tmem + lane_base + kDecTmemO, o);
+      }
+      if (warp < 2) {
+        // Lanes 0..63: head dim kl of every query row.
+        float* dst = p.o_part + cta * kDecRows * kHeadDim + kl;
+#pragma unroll
+        for (int n = 0; n < kR; ++n)
+          if (n < p.R) dst[n * kHeadDim] = have ? __uint_as_float(o[n]) : 0.f;
+      } else if (kl == 64) {
+        // Lane 64: the row sums.
+#pragma unroll
+        for (int n = 0; n < kR; ++n)
+          if (n < p.R) p.l_part[cta * kDecRows + n] = have ? __uint_as_float(o[n]) : 0.f;
+      }
+    }
+    if (kl < p.R) p.m_part[cta * kDecRows + kl] = (w.n > 0) ? ctl->m_ref[kl] : -INFINITY;
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kDecMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kDecTmemCols);
+  }
+}
+
+// Merges the splits of every (sequence, new token, query head) and adds the
+// sink: m = max(s, m_k), l = e^{s-m} + sum_k l_k e^{m_k-m},
+// out = sum_k O_k e^{m_k-m} / l, lse = m + ln l (exponents in base 2 here).
+// One warp per output row, two head dims per lane.
+__global__ void __launch_bounds__(128) sink_attn_decode_combine_kernel(const DecParams p, __nv_bfloat16* out,
+                                                                       float* lse) {
+  const int row = blockIdx.x * 4 + (threadIdx.x >> 5);  // (b * Lq + t) * Hq + h
+  const int lane = threadIdx.x & 31;
+  const int total = p.batch * p.Lq * p.Hq;
+  if (row >= total) return;
+  const int h = row % p.Hq;
+  const int bt = row / p.Hq;
+  const int b = bt / p.Lq;
+  const int t = bt % p.Lq;
+  const int g = h >> p.G_log2;
+  const int n = (t << p.G_log2) + (h & (p.G - 1));
+  const size_t base = (static_cast<size_t>(b) * p.Hkv + g) * p.n_split;
+  const float s2 = __ldg(p.sinks + h) * kLog2e;
+  float m = s2;
+  for (int k = 0; k < p.n_split; ++k) m = fmaxf(m, p.m_part[(base + k) * kDecRows + n]);
+  float l = 0.f, o0 = 0.f, o1 = 0.f;
+  if (m != -INFINITY) {
+    if (s2 != -INFINITY) l = ex2_approx(s2 - m);
+    for (int k = 0; k < p.n_split; ++k) {
+      const float mk = p.m_part[(base + k) * kDecRows + n];
+      if (mk == -INFINITY) continue;
+      const float f = ex2_approx(mk - m);
+      l = fmaf(p.l_part[(base + k) * kDecRows + n], f, l);
+      const float2 v = reinterpret_cast<const float2*>(p.o_part + ((base + k) * kDecRows + n) * kHeadDim)[lane];
+      o0 = fmaf(v.x, f, o0);
+      o1 = fmaf(v.y, f, o1);
+    }
+  }
+  const float inv = l > 0.f ? 1.f / l : 0.f;
+  reinterpret_cast<uint32_t*>(out + static_cast<size_t>(row) * kHeadDim)[lane] = pack_bf16x2(o0 * inv, o1 * inv);
+  if (lane == 0) lse[static_cast<size_t>(h) * (p.batch * p.Lq) + bt] = l > 0.f ? (m + __log2f(l)) * kLn2 : -INFINITY;
+}
+
+// Writes the new tokens' keys and values into their cache slots: token t of
+// sequence b goes to slot (cache_seqlens[b] + t) mod C.  One thread per 16
+// bytes.
+__global__ void __launch_bounds__(256) sink_attn_cache_append_kernel(const DecParams p, const uint4* k_new,
+                                                                     const uint4* v_new, uint4* k_cache,
+                                                                     uint4* v_cache) {
+  constexpr int kChunks = kHeadDim * 2 / 16;  // 16-byte chunks per [D] row
+  const long long total = static_cast<long long>(p.batch) * p.Lq * p.Hkv * kChunks;
+  const long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= 2 * total) return;
+  const bool is_v = i >= total;
+  const long long e = is_v ? i - total : i;
+  const int c = static_cast<int>(e % kChunks);
+  const long long r = e / kChunks;  // (b * Lq + t) * Hkv + g
+  const int g = static_cast<int>(r % p.Hkv);
+  const long long bt = r / p.Hkv;
+  const int b = static_cast<int>(bt / p.Lq);
+  const int t = static_cast<int>(bt % p.Lq);
+  const int L0 = __ldg(p.seqlens + b);
+  if (L0 < 0) return;  // reported by the attention kernel
+  const int slot = (L0 + t) % p.C;
+  const size_t dst = ((static_cast<size_t>(b) * p.C + slot) * p.Hkv + g) * kChunks + c;
+  if (is_v) v_cache[dst] = v_new[e];
+  else k_cache[dst] = k_new[e];
+}
+
+}  // namespace sa

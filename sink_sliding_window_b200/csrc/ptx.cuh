@@ -17,6 +17,10 @@ enum DeviceError : int {
   kDevErrTimeoutSoftmax = 0x103,
   kDevErrTimeoutEpilogue = 0x104,
   kDevErrTimeoutBwd = 0x105,
+  kDevErrTimeoutDecode = 0x106,
+  // A decode query needs a key whose cache slot already holds a newer
+  // token (the ring is smaller than window + new tokens - 1).
+  kDevErrDecodeCacheTooSmall = 0x201,
 };
 
 // One second: far beyond any legitimate wait in these kernels.

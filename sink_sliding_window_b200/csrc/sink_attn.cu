@@ -4,6 +4,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -15,6 +16,7 @@
 #include "tma_host.cuh"
 #include "fwd_kernel.cuh"
 #include "bwd_kernels.cuh"
+#include "decode_kernel.cuh"
 
 namespace sa {
 namespace {
@@ -74,6 +76,63 @@ bool set_smem_once(K kernel, size_t bytes, int* done_flag) {
     return false;
   *done_flag = 1;
   return true;
+}
+
+// Decode: sizes, split count and workspace layout of one call.
+struct DecPlan {
+  DecParams p;
+  size_t o_off, m_off, l_off, total;  // workspace layout (bytes)
+};
+
+// CTAs the split count aims for: two per SM of a 148-SM B200.
+constexpr int kDecTargetCtas = 296;
+
+size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
+
+sink_attn_status plan_decode(const sink_attn_decode_dims* d, int window, float scale, DecPlan* plan) {
+  if (!d) return SINK_ATTN_ERR_NULL;
+  if (d->batch < 0 || d->new_tokens <= 0 || d->cache_capacity <= 0 || d->max_seqlen < d->new_tokens ||
+      d->num_q_heads <= 0 || d->num_kv_heads <= 0 || d->head_dim <= 0)
+    return SINK_ATTN_ERR_SHAPE;
+  if (d->num_q_heads % d->num_kv_heads != 0) return SINK_ATTN_ERR_SHAPE;
+  if (d->head_dim != kHeadDim) return SINK_ATTN_ERR_UNSUPPORTED;
+  const int G = d->num_q_heads / d->num_kv_heads;
+  const int gl = ilog2_exact(G);
+  if (gl < 0 || static_cast<int64_t>(G) * d->new_tokens > kDecRows) return SINK_ATTN_ERR_UNSUPPORTED;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return SINK_ATTN_ERR_UNSUPPORTED;
+  // Slot and element indices are formed in 32-bit ints in places.
+  if (static_cast<int64_t>(d->batch) * d->cache_capacity > (int64_t(1) << 30) ||
+      static_cast<int64_t>(d->max_seqlen) + kDecTile > (int64_t(1) << 30) ||
+      static_cast<int64_t>(d->batch) * d->new_tokens * d->num_q_heads > (int64_t(1) << 30))
+    return SINK_ATTN_ERR_UNSUPPORTED;
+  DecParams& p = plan->p;
+  p.batch = d->batch;
+  p.Lq = d->new_tokens;
+  p.C = d->cache_capacity;
+  p.Hq = d->num_q_heads;
+  p.Hkv = d->num_kv_heads;
+  p.G = G;
+  p.G_log2 = gl;
+  p.R = G * d->new_tokens;
+  p.window = window > 0 ? window : 0;
+  p.scale_log2 = scale * kLog2e;
+  p.seqlens = nullptr;
+  p.sinks = nullptr;
+  p.o_part = p.m_part = p.l_part = nullptr;
+  // Upper bound on the 128-slot tiles one sequence scans.
+  int64_t slots = std::min<int64_t>(d->cache_capacity, d->max_seqlen);
+  if (p.window > 0) slots = std::min<int64_t>(slots, static_cast<int64_t>(p.window) + d->new_tokens - 1 + kDecTile);
+  const int tiles = static_cast<int>((slots + kDecTile - 1) / kDecTile) + 1;
+  const int64_t pairs = static_cast<int64_t>(d->batch) * d->num_kv_heads;
+  int split = pairs > 0 ? static_cast<int>((kDecTargetCtas + pairs - 1) / pairs) : 1;
+  split = std::max(1, std::min(split, std::max(1, tiles / 2)));
+  p.n_split = split;
+  const size_t parts = static_cast<size_t>(pairs) * split * kDecRows;
+  plan->o_off = 0;
+  plan->m_off = round256(parts * kHeadDim * sizeof(float));
+  plan->l_off = plan->m_off + round256(parts * sizeof(float));
+  plan->total = plan->l_off + round256(parts * sizeof(float));
+  return SINK_ATTN_OK;
 }
 
 }  // namespace
@@ -243,3 +302,68 @@ extern "C" sink_attn_status sink_attn_bwd_noalloc(const sink_attn_dims* d, const
   return sink_attn_bwd(d, q, k, v, sinks, cu_seqlens, window, scale, out, lse, dout, dq, dk, dv, dsinks, scratch,
                        SINK_ATTN_NOALLOC_SCRATCH_BYTES, stream);
 }
+
+extern "C" {
+
+size_t sink_attn_decode_workspace_size(const sink_attn_decode_dims* d, int window) {
+  DecPlan plan;
+  if (plan_decode(d, window, 1.f, &plan) != SINK_ATTN_OK) return 0;
+  return plan.total;
+}
+
+int sink_attn_decode_launches(const sink_attn_decode_dims* d) {
+  DecPlan plan;
+  if (plan_decode(d, 0, 1.f, &plan) != SINK_ATTN_OK) return 0;
+  return d->batch > 0 ? 3 : 0;
+}
+
+sink_attn_status sink_attn_decode(const sink_attn_decode_dims* d, const void* q, const void* k_new,
+                                  const void* v_new, void* k_cache, void* v_cache, const int* cache_seqlens,
+                                  const float* sinks, int window, float scale, void* out, float* lse,
+                                  void* workspace, size_t workspace_bytes, void* stream) {
+  DecPlan plan;
+  sink_attn_status st = plan_decode(d, window, scale, &plan);
+  if (st != SINK_ATTN_OK) return st;
+  if (d->batch == 0) return SINK_ATTN_OK;
+  if (!q || !k_new || !v_new || !k_cache || !v_cache || !cache_seqlens || !sinks || !out || !lse)
+    return SINK_ATTN_ERR_NULL;
+  if (!aligned16(q) || !aligned16(k_new) || !aligned16(v_new) || !aligned16(k_cache) || !aligned16(v_cache) ||
+      !aligned16(out) || (reinterpret_cast<uintptr_t>(lse) & 3u) || (reinterpret_cast<uintptr_t>(sinks) & 3u) ||
+      (reinterpret_cast<uintptr_t>(cache_seqlens) & 3u))
+    return SINK_ATTN_ERR_ALIGN;
+  if (!workspace || workspace_bytes < plan.total || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return SINK_ATTN_ERR_WORKSPACE;
+  DecParams p = plan.p;
+  p.seqlens = cache_seqlens;
+  p.sinks = sinks;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  p.o_part = reinterpret_cast<float*>(ws + plan.o_off);
+  p.m_part = reinterpret_cast<float*>(ws + plan.m_off);
+  p.l_part = reinterpret_cast<float*>(ws + plan.l_off);
+
+  CUtensorMap tq, tk, tv;
+  if (!make_map_3d(&tq, q, kHeadDim, p.Hq, p.batch * p.Lq, p.G, p.Lq) ||
+      !make_map_3d(&tk, k_cache, kHeadDim, p.Hkv, p.batch * p.C, 1, kDecTile) ||
+      !make_map_3d(&tv, v_cache, kHeadDim, p.Hkv, p.batch * p.C, 1, kDecTile))
+    return SINK_ATTN_ERR_CUDA;
+  // Register arrays sized for the real query rows.
+  void (*kern)(CUtensorMap, CUtensorMap, CUtensorMap, DecParams) =
+      p.R <= 16 ? sink_attn_decode_kernel<16> : (p.R <= 32 ? sink_attn_decode_kernel<32> : sink_attn_decode_kernel<64>);
+  static int smem_set[3] = {0, 0, 0};
+  if (!set_smem_once(kern, kDecSmemBytes, &smem_set[p.R <= 16 ? 0 : (p.R <= 32 ? 1 : 2)])) return SINK_ATTN_ERR_CUDA;
+  const long long ctas = static_cast<long long>(p.batch) * p.Hkv * p.n_split;
+  if (ctas > 0x7fffffff) return SINK_ATTN_ERR_UNSUPPORTED;
+
+  cudaStream_t st_ = static_cast<cudaStream_t>(stream);
+  const long long chunks = 2LL * p.batch * p.Lq * p.Hkv * (kHeadDim * 2 / 16);
+  sink_attn_cache_append_kernel<<<static_cast<unsigned>((chunks + 255) / 256), 256, 0, st_>>>(
+      p, static_cast<const uint4*>(k_new), static_cast<const uint4*>(v_new), static_cast<uint4*>(k_cache),
+      static_cast<uint4*>(v_cache));
+  kern<<<static_cast<unsigned>(ctas), kDecThreads, kDecSmemBytes, st_>>>(tq, tk, tv, p);
+  const long long rows = static_cast<long long>(p.batch) * p.Lq * p.Hq;
+  sink_attn_decode_combine_kernel<<<static_cast<unsigned>((rows + 3) / 4), 128, 0, st_>>>(
+      p, static_cast<__nv_bfloat16*>(out), lse);
+  return cudaPeekAtLastError() == cudaSuccess ? SINK_ATTN_OK : SINK_ATTN_ERR_CUDA;
+}
+
+}  // extern "C"

@@ -26,7 +26,8 @@ STATUS = {
 }
 
 EXPORTS = ("sink_attn_fwd", "sink_attn_bwd", "sink_attn_bwd_workspace_size", "sink_attn_status_string",
-           "sink_attn_device_error", "sink_attn_fwd_launches", "sink_attn_bwd_launches", "sink_attn_profile_events")
+           "sink_attn_device_error", "sink_attn_fwd_launches", "sink_attn_bwd_launches", "sink_attn_profile_events",
+           "sink_attn_decode", "sink_attn_decode_workspace_size", "sink_attn_decode_launches")
 
 
 class SinkAttnError(RuntimeError):
@@ -38,6 +39,12 @@ class SinkAttnError(RuntimeError):
 class Dims(ctypes.Structure):
     _fields_ = [("batch", ctypes.c_int), ("max_seqlen", ctypes.c_int), ("total_tokens", ctypes.c_int),
                 ("num_q_heads", ctypes.c_int), ("num_kv_heads", ctypes.c_int), ("head_dim", ctypes.c_int)]
+
+
+class DecodeDims(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int), ("new_tokens", ctypes.c_int), ("cache_capacity", ctypes.c_int),
+                ("max_seqlen", ctypes.c_int), ("num_q_heads", ctypes.c_int), ("num_kv_heads", ctypes.c_int),
+                ("head_dim", ctypes.c_int)]
 
 
 def lib_path() -> str:
@@ -71,6 +78,13 @@ def load():
         L.sink_attn_bwd_launches.restype = I
         L.sink_attn_profile_events.argtypes = [I, P, P]
         L.sink_attn_profile_events.restype = I
+        DD = ctypes.POINTER(DecodeDims)
+        L.sink_attn_decode.argtypes = [DD, P, P, P, P, P, P, P, I, ctypes.c_float, P, P, P, ctypes.c_size_t, P]
+        L.sink_attn_decode.restype = I
+        L.sink_attn_decode_workspace_size.argtypes = [DD, I]
+        L.sink_attn_decode_workspace_size.restype = ctypes.c_size_t
+        L.sink_attn_decode_launches.argtypes = [DD]
+        L.sink_attn_decode_launches.restype = I
         _lib = L
     return _lib
 
@@ -154,6 +168,51 @@ def bwd(q, k, v, sinks, out, lse, dout, cu_seqlens=None, window=0, scale=None, *
     if st != 0:
         raise SinkAttnError(st, "sink_attn_bwd")
     return dq, dk, dv, dsinks
+
+
+def decode_dims(batch, new_tokens, cache_capacity, max_seqlen, Hq, Hkv, D=64) -> DecodeDims:
+    return DecodeDims(int(batch), int(new_tokens), int(cache_capacity), int(max_seqlen), int(Hq), int(Hkv), int(D))
+
+
+def decode_workspace_size(batch, new_tokens, cache_capacity, max_seqlen, Hq, Hkv, window=0, D=64) -> int:
+    d = decode_dims(batch, new_tokens, cache_capacity, max_seqlen, Hq, Hkv, D)
+    return int(load().sink_attn_decode_workspace_size(ctypes.byref(d), int(window)))
+
+
+def decode_launches(batch, new_tokens, cache_capacity, max_seqlen, Hq, Hkv, D=64) -> int:
+    d = decode_dims(batch, new_tokens, cache_capacity, max_seqlen, Hq, Hkv, D)
+    return int(load().sink_attn_decode_launches(ctypes.byref(d)))
+
+
+def decode(q, k_new, v_new, k_cache, v_cache, cache_seqlens, sinks, window=0, scale=None, *, max_seqlen=None,
+           out=None, lse=None, workspace=None, stream=None):
+    """sink_attn_decode.  q [B, Lq, Hq, D], k_new / v_new [B, Lq, Hkv, D],
+    k_cache / v_cache [B, C, Hkv, D] (bf16, CUDA; the new tokens are written
+    into the cache), cache_seqlens int32 [B] CUDA (tokens cached before this
+    call; not modified), sinks [Hq] fp32.  max_seqlen bounds
+    cache_seqlens + Lq (default: C + Lq).  Returns (out [B, Lq, Hq, D],
+    lse [Hq, B * Lq])."""
+    B, Lq, Hq, D = q.shape
+    C, Hkv = k_cache.shape[1], k_cache.shape[2]
+    if max_seqlen is None:
+        max_seqlen = C + Lq
+    if scale is None:
+        scale = D ** -0.5
+    dims = decode_dims(B, Lq, C, max_seqlen, Hq, Hkv, D)
+    L = load()
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((Hq, B * Lq), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        need = int(L.sink_attn_decode_workspace_size(ctypes.byref(dims), int(window)))
+        workspace = torch.empty((max(need, 1),), dtype=torch.uint8, device=q.device)
+    st = L.sink_attn_decode(ctypes.byref(dims), _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache),
+                            _ptr(cache_seqlens), _ptr(sinks), int(window), float(scale), _ptr(out), _ptr(lse),
+                            _ptr(workspace), ctypes.c_size_t(workspace.numel()), _stream_handle(stream))
+    if st != 0:
+        raise SinkAttnError(st, "sink_attn_decode")
+    return out, lse
 
 
 def device_error(stream=None) -> int:

@@ -20,7 +20,8 @@ from dataclasses import dataclass, field
 
 import numpy as np
 
-_IDS = {"q": 1, "k": 2, "v": 3, "sinks": 4, "dout": 5, "doclens": 6, "rows": 7}
+_IDS = {"q": 1, "k": 2, "v": 3, "sinks": 4, "dout": 5, "doclens": 6, "rows": 7,
+        "dec_q": 11, "dec_k": 12, "dec_v": 13, "dec_sinks": 14}
 
 
 def _rng(seed: int, name: str) -> np.random.Generator:
@@ -137,3 +138,23 @@ def workload(name: str, seed: int = 0) -> Workload:
 
 WORKLOADS = ["tiny:w32", "tiny:full", "prefill4k:w128", "prefill4k:full", "varlen64k:w128",
              "varlen64k:full", "long60k:full", "long60k:w128"]
+
+
+def decode_inputs(seed: int, cached: list, new_tokens: int, Hq: int, Hkv: int, D: int = 64,
+                  sink_std: float = 1.0) -> dict:
+    """Seeded inputs of one decode call (gpt-oss head shapes by default).
+
+    Sequence b has `cached[b]` tokens before the call and `new_tokens` new
+    ones.  Returns the whole token history of every sequence packed one after
+    another -- k, v [T][Hkv][D] bf16 bits with cu [B+1] -- the new tokens'
+    queries q_new [B][new_tokens][Hq][D] (bf16 bits) and sinks [Hq] fp32.
+    The new tokens of sequence b are history positions cached[b] ..
+    cached[b] + new_tokens - 1."""
+    lens = [int(c) + int(new_tokens) for c in cached]
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    T = int(cu[-1])
+    s = _rng(seed, "dec_sinks").standard_normal(size=(Hq,), dtype=np.float32) * np.float32(sink_std)
+    return dict(k=normal_bf16(seed, "dec_k", (T, Hkv, D)), v=normal_bf16(seed, "dec_v", (T, Hkv, D)),
+                q_new=normal_bf16(seed, "dec_q", (len(cached), new_tokens, Hq, D)),
+                sinks=s.astype(np.float32), cu=cu)
+

@@ -105,3 +105,52 @@ def test_launch_counts(L):
     assert L.sink_attn_fwd_launches(ctypes.byref(dims())) == 1
     assert L.sink_attn_fwd_launches(ctypes.byref(dims(T=0, batch=0, max_seqlen=0))) == 0
     assert L.sink_attn_bwd_launches(ctypes.byref(dims())) >= 0
+
+
+def ddims(B=4, Lq=1, C=256, max_seqlen=257, Hq=64, Hkv=8, D=64):
+    return ops.decode_dims(B, Lq, C, max_seqlen, Hq, Hkv, D)
+
+
+def call_decode(L, d, ptrs=None, window=0, scale=0.125, ws=FAKE, ws_bytes=1 << 30):
+    # q, k_new, v_new, k_cache, v_cache, cache_seqlens, sinks, window, scale, out, lse, workspace, bytes, stream
+    p = [FAKE] * 7 if ptrs is None else ptrs
+    return L.sink_attn_decode(ctypes.byref(d), *p[:7], int(window), ctypes.c_float(scale), FAKE, FAKE, ws,
+                              ctypes.c_size_t(ws_bytes), None)
+
+
+def test_decode_workspace_size(L):
+    w = ops.decode_workspace_size(4, 1, 8192, 8192, 64, 8)
+    assert w > 0 and w % 256 == 0
+    # Partials for at least one split of 64 query rows x 64 dims per (sequence, kv head).
+    assert w >= 4 * 8 * 64 * 64 * 4
+    assert ops.decode_workspace_size(4, 1, 8192, 8192, 64, 8, D=32) == 0
+    assert ops.decode_workspace_size(4, 9, 8192, 8192, 64, 8) == 0  # G * Lq = 72 > 64
+
+
+@pytest.mark.parametrize("bad,code", [
+    (dict(Lq=0), 2), (dict(C=0), 2), (dict(B=-1), 2), (dict(max_seqlen=0), 2), (dict(Hq=63), 2),
+    (dict(D=128), 4), (dict(Hq=48, Hkv=8), 4), (dict(Lq=9), 4),
+])
+def test_decode_rejects_bad_sizes(L, bad, code):
+    assert call_decode(L, ddims(**bad)) == code
+
+
+def test_decode_rejects_bad_pointers_scale_and_workspace(L):
+    d = ddims()
+    for i in range(7):
+        p = [FAKE] * 7
+        p[i] = None
+        assert call_decode(L, d, p) == 1, i
+    p = [FAKE] * 7
+    p[3] = ctypes.c_void_p((1 << 20) + 8)  # k_cache misaligned
+    assert call_decode(L, d, p) == 3
+    assert call_decode(L, d, scale=0.0) == 4
+    need = ops.decode_workspace_size(4, 1, 256, 257, 64, 8)
+    assert call_decode(L, d, ws_bytes=need - 1) == 7
+    assert call_decode(L, d, ws=None) == 7
+
+
+def test_decode_empty_batch_is_noop(L):
+    assert call_decode(L, ddims(B=0), [None] * 7, ws=None, ws_bytes=0) == 0
+    assert ops.decode_launches(0, 1, 256, 257, 64, 8) == 0
+    assert ops.decode_launches(4, 1, 256, 257, 64, 8) == 3

@@ -1,0 +1,152 @@
+"""sink_attn_decode (CUDA, through the C ABI) against the fp64 oracle.
+
+Decode evaluates the forward definition at the newest positions of each
+sequence, so the oracle is the forward itself: every sequence's whole token
+history is packed as one document per sequence and oracle.fwd_rows evaluates
+the rows of the new tokens.  The GPU sees the same tokens through its cache:
+history position p < L0 sits in slot p mod C (later positions overwrite
+earlier ones, so a ring keeps the last C), the new tokens are passed
+separately and appended by the call.  Slots that hold no token are filled
+with NaN: no result may depend on them.  Tolerances: 1e-2 (out) and 1e-3
+(lse) of the oracle tensor's max-abs."""
+import numpy as np
+import pytest
+
+import oracle
+from sink_sliding_window_b200 import synth
+from tests.gpu_util import TOL_LSE, TOL_OUT, check, dev, dev_bf16, host_f64
+
+pytestmark = pytest.mark.gpu
+
+NAN_BF16 = np.uint16(0x7FC0)
+SCALE = 0.125
+
+
+@pytest.fixture(scope="module")
+def ops():
+    import torch
+    from sink_sliding_window_b200 import build, ops as _ops
+    assert torch.cuda.is_available()
+    build.build()
+    return _ops
+
+
+def _cache_from_history(hist, cu, cached, C):
+    """[B][C][H][D] cache holding positions p < cached[b] at slot p mod C;
+    untouched slots are NaN."""
+    B = len(cached)
+    H, D = hist.shape[1], hist.shape[2]
+    cache = np.full((B, C, H, D), NAN_BF16, np.uint16)
+    for b in range(B):
+        for p in range(int(cached[b])):
+            cache[b, p % C] = hist[int(cu[b]) + p]
+    return cache
+
+
+def _oracle_rows(a, cached, Lq, window, seqs=None):
+    """Oracle out / lse for the new tokens of the sequences `seqs` (all by
+    default), one sequence at a time (each sequence is its own document)."""
+    cu = a["cu"]
+    seqs = range(len(cached)) if seqs is None else seqs
+    Hq, D = a["q_new"].shape[2], a["q_new"].shape[3]
+    outs, lses = [], []
+    for b in seqs:
+        lo, hi = int(cu[b]), int(cu[b + 1])
+        L = hi - lo
+        q = np.zeros((L, Hq, D), np.uint16)
+        q[int(cached[b]):] = a["q_new"][b]
+        rows = np.arange(int(cached[b]), L, dtype=np.int64)
+        o, l = oracle.fwd_rows(q, a["k"][lo:hi], a["v"][lo:hi], a["sinks"], np.array([0, L], np.int32), window,
+                               SCALE, rows)
+        outs.append(o)
+        lses.append(l)
+    return np.concatenate(outs), np.concatenate(lses, axis=1)
+
+
+def _run(ops, cached, Lq, Hq, Hkv, C, window, seed, sinks=None, check_all=True, seqs=None):
+    import torch
+    a = synth.decode_inputs(seed, cached, Lq, Hq, Hkv)
+    if sinks is not None:
+        a["sinks"] = np.asarray(sinks, np.float32)
+    cu = a["cu"]
+    B = len(cached)
+    kc0 = _cache_from_history(a["k"], cu, cached, C)
+    vc0 = _cache_from_history(a["v"], cu, cached, C)
+    new_idx = np.concatenate([np.arange(int(cu[b]) + int(cached[b]), int(cu[b + 1])) for b in range(B)])
+    k_new = a["k"][new_idx].reshape(B, Lq, Hkv, 64)
+    v_new = a["v"][new_idx].reshape(B, Lq, Hkv, 64)
+    kc, vc = dev_bf16(kc0), dev_bf16(vc0)
+    seqlens = dev(np.asarray(cached, np.int32))
+    out, lse = ops.decode(dev_bf16(a["q_new"]), dev_bf16(k_new), dev_bf16(v_new), kc, vc, seqlens,
+                          dev(a["sinks"]), window, SCALE, max_seqlen=int(max(cached)) + Lq)
+    torch.cuda.synchronize()
+    assert ops.device_error() == 0
+    # The new tokens are in their slots; nothing else changed (bitwise).
+    ke, ve = kc0.copy(), vc0.copy()
+    for b in range(B):
+        for t in range(Lq):
+            ke[b, (int(cached[b]) + t) % C] = k_new[b, t]
+            ve[b, (int(cached[b]) + t) % C] = v_new[b, t]
+    assert np.array_equal(kc.view(torch.int16).cpu().numpy().view(np.uint16), ke), "k cache after append"
+    assert np.array_equal(vc.view(torch.int16).cpu().numpy().view(np.uint16), ve), "v cache after append"
+    seqs = list(range(B)) if seqs is None else list(seqs)
+    ro, rl = _oracle_rows(a, cached, Lq, window, seqs)
+    got_o = host_f64(out)[seqs].reshape(-1, Hq, 64)
+    got_l = host_f64(lse).reshape(Hq, B, Lq)[:, seqs].reshape(Hq, -1)
+    eo = check(got_o, ro, TOL_OUT, "decode out")
+    el = check(got_l, rl, TOL_LSE, "decode lse")
+    return eo, el
+
+
+@pytest.mark.parametrize("window", [0, 100])
+def test_linear_cache_one_token(ops, window):
+    """One new token, a linear cache (C >= every length), lengths across tile
+    edges, including an empty cache."""
+    _run(ops, [0, 1, 99, 127, 128, 129, 300, 1000], 1, 16, 2, 1152, window, seed=1)
+
+
+@pytest.mark.parametrize("Lq", [1, 2, 5])
+def test_ring_cache_window(ops, Lq):
+    """Sliding-window layer on a ring of exactly window + Lq - 1 slots,
+    before and after the ring wraps."""
+    W = 128
+    _run(ops, [0, 5, 126, 127, 128, 129, 200, 1000], Lq, 16, 2, W + Lq - 1, W, seed=2 + Lq)
+
+
+def test_small_window_ring_several_tokens(ops):
+    """Window 16 on an 18-slot ring with 3 new tokens: the causal mask among
+    the new tokens and the window edge both matter."""
+    _run(ops, [0, 2, 17, 40, 333], 3, 16, 2, 18, 16, seed=7)
+
+
+@pytest.mark.parametrize("G,Lq", [(1, 1), (4, 2), (8, 4), (16, 4)])
+def test_group_sizes_and_rows(ops, G, Lq):
+    """G x Lq query rows per head group from 1 to 64 (every register-tile
+    variant of the kernel)."""
+    _run(ops, [0, 64, 257], Lq, 2 * G, 2, 512, 0, seed=10 + G)
+
+
+def test_sink_extremes(ops):
+    sinks = [-np.inf, -1e4, 0.0, 1e4, 0.5, -0.5, 3.0, -np.inf]
+    for window, C in ((0, 640), (64, 64)):
+        _run(ops, [0, 1, 63, 64, 600], 1, 8, 1, C, window, seed=20, sinks=sinks)
+
+
+def test_wide_cache_with_window_skips_old_slots(ops):
+    """A linear cache much longer than the window: only the slot tiles the
+    window reaches are visited."""
+    _run(ops, [50, 1500, 4000], 1, 16, 2, 4200, 100, seed=30)
+
+
+@pytest.mark.parametrize("window,C", [(0, 8192), (128, 128)])
+def test_gpt_oss_decode_full_size(ops, window, C):
+    """gpt-oss heads (Hq 64, Hkv 8), 64 sequences at 8191 cached tokens plus
+    one new token: full-causal layer on a linear cache and window-128 layer
+    on a 128-slot ring; the oracle checks 6 of the 64 sequences, all heads."""
+    cached = [8191] * 62 + [0, 4000]
+    _run(ops, cached, 1, 64, 8, C, window, seed=40, seqs=[0, 1, 31, 61, 62, 63])
+
+
+def test_launch_count(ops):
+    assert ops.decode_launches(4, 1, 256, 257, 64, 8) == 3
+    assert ops.decode_launches(0, 1, 256, 257, 64, 8) == 0
