@@ -196,6 +196,61 @@ def measured_traffic():
     return t.get("dram_bytes_per_launch") if t.get("kernel_source_hash") == kernel_source_hash() else None
 
 
+# --------------------------------------------------------------- decode
+DECODE_CASES = (
+    # (name, sequences, cached tokens, new tokens, cache slots, window)
+    ("decode 64 seqs x 8191 cached + 1 new, full-causal layer, linear 8192-slot cache", 64, 8191, 1, 8192, 0),
+    ("decode 64 seqs x 8191 cached + 1 new, window-128 layer, 128-slot ring", 64, 8191, 1, 128, 128),
+)
+
+
+def measure_decode(torch, ops, stream, iters=20):
+    """Times sink_attn_decode (append + attend + combine) on gpt-oss heads with
+    CUDA events on the launching stream, writing a 256 MiB buffer between
+    iterations so that no K/V tile is served from L2.  Bandwidth counts the
+    K and V bytes the new queries must read (every cached key they can see)."""
+    _, hbm, kind = read_peaks()
+    res = []
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    for name, Bd, L0, Lq, C, W in DECODE_CASES:
+        a = synth.decode_inputs(7, [0], Lq, HQ, HKV)  # sinks and new-token rows
+        g = torch.Generator(device="cuda").manual_seed(7)
+        mk = lambda *shape: torch.randn(*shape, device="cuda", generator=g).to(torch.bfloat16)  # noqa: E731
+        q, kn, vn = mk(Bd, Lq, HQ, D), mk(Bd, Lq, HKV, D), mk(Bd, Lq, HKV, D)
+        kc, vc = mk(Bd, C, HKV, D), mk(Bd, C, HKV, D)
+        sl = torch.full((Bd,), L0, dtype=torch.int32, device="cuda")
+        sinks = torch.from_numpy(a["sinks"]).cuda()
+        ws = torch.empty((ops.decode_workspace_size(Bd, Lq, C, L0 + Lq, HQ, HKV, W),), dtype=torch.uint8,
+                         device="cuda")
+        out = torch.empty_like(q)
+        lse = torch.empty((HQ, Bd * Lq), dtype=torch.float32, device="cuda")
+
+        def call():
+            ops.decode(q, kn, vn, kc, vc, sl, sinks, W, 0.125, max_seqlen=L0 + Lq, out=out, lse=lse, workspace=ws,
+                       stream=stream)
+        for _ in range(3):
+            call()
+        torch.cuda.synchronize()
+        tot = 0.0
+        for _ in range(iters):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            call()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            tot += e0.elapsed_time(e1)
+        if ops.device_error() != 0:
+            raise RuntimeError("a decode kernel reported an error")
+        ms = tot / iters
+        keys = min(L0 + Lq, C) if W <= 0 else min(L0 + Lq, W + Lq - 1, C)
+        kv = Bd * keys * HKV * D * 2 * 2
+        res.append({"workload": name, "us": ms * 1e3, "kv_bytes": kv, "achieved_GBps": kv / ms / 1e6,
+                    "peak_GBps": hbm, "frac": kv / ms / 1e6 / hbm, "peak_source": f"{kind} hbm_gbs",
+                    "launches": ops.decode_launches(Bd, Lq, C, L0 + Lq, HQ, HKV)})
+    return res
+
+
 # ----------------------------------------------------------- aggregation
 def max_over_ranks(x, dist, device):
     """Largest value of x over all ranks (the slowest rank's time); x itself
@@ -350,6 +405,8 @@ def run_ours(args, rank, world, torch, dist):
     e2e_ms = max_over_ranks(x0.elapsed_time(x1), dist, "cuda")
     e2e_value = job_throughput(world, flops, e2e_steps, e2e_ms)
 
+    decode = measure_decode(torch, ops, stream) if not args.skip_decode else None
+
     if rank != 0:
         return
     peak, _, peak_kind = read_peaks()
@@ -370,6 +427,8 @@ def run_ours(args, rank, world, torch, dist):
         "gpu_launches": launches,
         "clocks": clk,
     }
+    if decode is not None:
+        line["decode"] = decode
     if world == 1 and not args.skip_cpu_baseline:
         secs, cflops, desc, threads = oracle_sample(S, 2048)
         line["cpu_baseline"] = {"value": cflops / secs / 1e12, "unit": "TFLOP/s", "cores": threads,
@@ -385,6 +444,7 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--skip-cpu-baseline", action="store_true")
+    ap.add_argument("--skip-decode", action="store_true", help="do not time sink_attn_decode after the step")
     ap.add_argument("--budget-s", type=float, default=120.0,
                     help="--impl reference: seconds all warmup + timed oracle steps should take")
     args = ap.parse_args(argv)

@@ -84,8 +84,10 @@ struct DecPlan {
   size_t o_off, m_off, l_off, total;  // workspace layout (bytes)
 };
 
-// CTAs the split count aims for: two per SM of a 148-SM B200.
+// CTAs that run at once (two per SM of a 148-SM B200), and a cap on the
+// splits of one (sequence, key/value head).
 constexpr int kDecTargetCtas = 296;
+constexpr int kDecMaxSplit = 64;
 
 size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
 
@@ -124,8 +126,22 @@ sink_attn_status plan_decode(const sink_attn_decode_dims* d, int window, float s
   if (p.window > 0) slots = std::min<int64_t>(slots, static_cast<int64_t>(p.window) + d->new_tokens - 1 + kDecTile);
   const int tiles = static_cast<int>((slots + kDecTile - 1) / kDecTile) + 1;
   const int64_t pairs = static_cast<int64_t>(d->batch) * d->num_kv_heads;
-  int split = pairs > 0 ? static_cast<int>((kDecTargetCtas + pairs - 1) / pairs) : 1;
-  split = std::max(1, std::min(split, std::max(1, tiles / 2)));
+  // Split count: the CTAs run in waves of kDecTargetCtas, each CTA over
+  // ceil(tiles / split) tiles plus about one tile's worth of fixed cost
+  // (set-up, Q load, partial results); pick the split with the fewest
+  // tile-times, preferring fewer splits on ties.
+  int split = 1;
+  if (pairs > 0) {
+    int64_t best = -1;
+    for (int k = 1; k <= std::min(tiles, kDecMaxSplit); ++k) {
+      const int64_t waves = (pairs * k + kDecTargetCtas - 1) / kDecTargetCtas;
+      const int64_t cost = waves * ((tiles + k - 1) / k + 1);
+      if (best < 0 || cost < best) {
+        best = cost;
+        split = k;
+      }
+    }
+  }
   p.n_split = split;
   const size_t parts = static_cast<size_t>(pairs) * split * kDecRows;
   plan->o_off = 0;
