@@ -208,6 +208,27 @@ sink_attn_status sink_attn_decode(const sink_attn_decode_dims* dims,
                                   void* workspace, size_t workspace_bytes,
                                   void* stream);
 
+/* Decode over an FP8 (e4m3) cache.  As sink_attn_decode(), except that
+ * k_cache / v_cache hold e4m3 codes, one byte per element,
+ * [batch][C][Hkv][D], with one dequantisation scale per key/value head:
+ * key = code * k_scale[g], value = code * v_scale[g] (k_scale, v_scale:
+ * fp32 [Hkv], device, > 0).  The pages list FP8 training recipes (Megatron-LM
+ * issue 1739 and its example scripts); this is the place on this path where
+ * FP8 pays on B200 at head dim 64: decode is HBM-bound, and e4m3 storage
+ * halves the bytes the cache moves, while the MMAs stay bf16 (e4m3 values
+ * are exact in bf16).  The call quantises the new tokens' k_new / v_new
+ * (bf16) as code = e4m3(x * (1 / scale)), rounded to nearest even and
+ * saturated to +-448, into their slots.  The workspace size is that of
+ * sink_attn_decode_workspace_size(). */
+sink_attn_status sink_attn_decode_e4m3(const sink_attn_decode_dims* dims,
+                                       const void* q, const void* k_new, const void* v_new,
+                                       void* k_cache, void* v_cache, const int* cache_seqlens,
+                                       const float* k_scale, const float* v_scale,
+                                       const float* sinks, int window, float scale,
+                                       void* out, float* lse,
+                                       void* workspace, size_t workspace_bytes,
+                                       void* stream);
+
 /* Number of kernels one sink_attn_decode call launches (0 when batch = 0). */
 int sink_attn_decode_launches(const sink_attn_decode_dims* dims);
 

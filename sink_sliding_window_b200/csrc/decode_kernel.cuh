@@ -29,23 +29,41 @@
 // slot order; each key's position (and so its mask) follows from the slot.
 // Each split writes (O, l, m) partials; the combine kernel merges them and
 // adds the sink's e^{s-m} once.
+//
+// e4m3 cache variant (kF8): the cache holds FP8 e4m3 codes with one
+// dequantisation scale per key/value head (k = code * k_scale[g], likewise
+// v).  Tiles arrive as bytes; the softmax threads (one slot each) widen their
+// slot's K row straight into TMEM, where it is the A operand of the S^T MMA,
+// and their V row into a shared-memory tile for the PV MMA.  This variant's
+// MMAs run in fp16: one instruction widens two e4m3 codes to fp16, exactly;
+// Q is converted from bf16 to fp16 once per CTA (saturating at +-65504) and P
+// is rounded to fp16 (P <= 2^8 here, so fp16 keeps more of it than bf16).
+// k_scale folds into the logit scale and v_scale into O.  Half the bytes of
+// the bf16 cache cross HBM.
 #pragma once
+#include <cuda_fp16.h>
+
 #include "common.cuh"
 
 namespace sa {
 
 constexpr int kDecThreads = 192;  // warps 0-3 softmax (one key per thread), 4 TMA producer, 5 MMA
+constexpr int kDecThreads8 = 320; // e4m3 cache: + warps 6-9 widening K and V (one slot per thread)
+constexpr int kDecConvWarp0 = 6;
 constexpr int kDecProducerWarp = 4;
 constexpr int kDecMmaWarp = 5;
 constexpr int kDecRows = 64;      // MMA N: query rows per CTA (G x Lq <= 64)
 constexpr int kDecTile = 128;     // slots per key tile (MMA M)
-constexpr int kDecStages = 2;
+constexpr int kDecStages = 2;      // bf16 cache: K/V tile stages
+constexpr int kDecStages8 = 3;     // e4m3 cache: byte-tile stages
 constexpr int kDecQBytes = kDecRows * kHeadDim * 2;    // Q tile, [64][64] bf16
 constexpr int kDecKvBytes = kDecTile * kHeadDim * 2;   // one K or V tile, [128][64] bf16
 constexpr int kDecPBytes = kDecTile * kDecRows * 2;    // P^T tile, [128 keys][64 rows] bf16
+constexpr int kDecKv8Bytes = kDecTile * kHeadDim;      // one e4m3 K or V tile, [128][64] bytes
 constexpr uint32_t kDecTmemCols = 256;  // S^T buffers [0,64), [64,128); O^T [128,192)
 constexpr uint32_t kDecTmemS = 0;
 constexpr uint32_t kDecTmemO = 128;
+constexpr uint32_t kDecTmemK = 192;  // e4m3 cache: widened K tiles, two 32-column buffers
 constexpr float kDecRescaleLog2 = 8.0f;
 
 struct DecParams {
@@ -55,6 +73,8 @@ struct DecParams {
   int n_split;                      // CTAs per (sequence, kv head)
   float scale_log2;                 // scale * log2(e)
   const int* seqlens;               // [batch] tokens in the cache before this call
+  const float* k_scale;             // e4m3 cache: [Hkv] dequantisation scales (else unused)
+  const float* v_scale;
   const float* sinks;               // [Hq]
   float* o_part;                    // [batch][Hkv][n_split][64 rows][64] unnormalised O
   float* m_part;                    // [batch][Hkv][n_split][64 rows] reference max (log2 units)
@@ -63,10 +83,13 @@ struct DecParams {
 
 struct DecCtl {
   uint64_t q_full;
-  uint64_t k_full[kDecStages];
-  uint64_t k_empty[kDecStages];
-  uint64_t v_full[kDecStages];
-  uint64_t v_empty[kDecStages];
+  uint64_t q_conv;      // e4m3 cache: Q converted to fp16 in place (128 arrivals)
+  uint64_t k_full[kDecStages8];
+  uint64_t k_empty[kDecStages8];
+  uint64_t v_full[kDecStages8];
+  uint64_t v_empty[kDecStages8];
+  uint64_t kt_full[2];  // e4m3 cache: K of tile i widened into TMEM buffer i % 2 (128 arrivals)
+  uint64_t v_ready;     // e4m3 cache: V of tile i widened into the fp16 tile (128 arrivals)
   uint64_t s_full[2];   // S^T of tile i in TMEM buffer i % 2
   uint64_t s_free[2];   // the softmax has loaded that S^T (128 arrivals)
   uint64_t p_full;      // P^T of tile i written (128 arrivals)
@@ -83,6 +106,8 @@ struct DecCtl {
 
 constexpr size_t kDecSmemBytes = 1024 /*alignment slack*/ + kDecQBytes + 2 * kDecStages * kDecKvBytes +
                                  kDecKvBytes /*ones*/ + kDecPBytes + sizeof(DecCtl);
+constexpr size_t kDecSmemBytes8 = 1024 + kDecQBytes + 2 * kDecStages8 * kDecKv8Bytes + kDecKvBytes /*bf16 V*/ +
+                                  kDecKvBytes /*ones*/ + kDecPBytes + sizeof(DecCtl);
 
 // Slot range of one CTA: [z0, z0 + 128 n) in 128-slot tiles.
 struct DecWork {
@@ -147,13 +172,54 @@ __device__ __forceinline__ void dec_issue_qk(uint32_t tmem_s, uint32_t k_addr, u
   }
 }
 
+// S^T = K Q^T in fp16 with K (32 packed columns) read from TMEM.
+__device__ __forceinline__ void dec_issue_qk_ts(uint32_t tmem_s, uint32_t tmem_k, uint32_t q_addr) {
+  constexpr uint32_t idesc = make_idesc_f16(kDecTile, kDecRows, 0, 0);
+#pragma unroll
+  for (int kk = 0; kk < kHeadDim / 16; ++kk) {
+    const uint64_t b = make_sdesc_sw128(q_addr + kk * 32, 16, 1024);
+    mma_ts(tmem_s, tmem_k + kk * 8, b, idesc, kk > 0 ? 1u : 0u);
+  }
+}
+
+// Two e4m3 codes (low byte first) -> two fp16 (low half first); exact.
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t codes) {
+  uint32_t h2;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(static_cast<uint16_t>(codes & 0xFFFFu)));
+  return h2;
+}
+
+// One cache row of 64 e4m3 codes -> 32 packed fp16 pairs (element order kept).
+__device__ __forceinline__ void dec_row_e4m3_to_f16(const uint8_t* src, uint32_t* out) {
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const uint4 v = reinterpret_cast<const uint4*>(src)[q];
+    const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      out[8 * q + 2 * u] = e4m3x2_to_f16x2(w4[u]);
+      out[8 * q + 2 * u + 1] = e4m3x2_to_f16x2(w4[u] >> 16);
+    }
+  }
+}
+
+// Two bf16 (packed) -> two fp16 (packed), rounded to nearest, saturating.
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2_sat(uint32_t v) {
+  const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&v));
+  uint32_t r;
+  asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(f.y), "f"(f.x));
+  return r;
+}
+
 // O^T (+)= [V | 1]^T P^T over the 128 slots of a tile: A (M = 128) is read
 // MN-major from the V tile (M rows 0..63) and the ones tile (M rows 64..127,
 // reached through the descriptor's leading-byte offset); B = P^T [slots][64
 // rows], MN-major.
+template <bool kF16>
 __device__ __forceinline__ void dec_issue_pv(uint32_t tmem_o, uint32_t v_addr, uint32_t ones_addr, uint32_t p_addr,
                                              bool accumulate) {
-  constexpr uint32_t idesc = make_idesc_bf16(kDecTile, kDecRows, 1, 1);
+  constexpr uint32_t idesc =
+      kF16 ? make_idesc_f16(kDecTile, kDecRows, 1, 1) : make_idesc_bf16(kDecTile, kDecRows, 1, 1);
   const uint32_t lbo = ones_addr - v_addr;
 #pragma unroll
   for (int kk = 0; kk < kDecTile / 16; ++kk) {
@@ -188,15 +254,20 @@ __device__ __forceinline__ void dec_tmem_st(uint32_t taddr, const uint32_t* r) {
 }
 
 // kR: query rows handled in registers (16, 32 or 64; >= G * Lq).
-template <int kR>
-__global__ void __launch_bounds__(kDecThreads, 2)
+// kF8: the cache holds e4m3 codes (see the file comment).
+template <int kR, bool kF8>
+__global__ void __launch_bounds__(kF8 ? kDecThreads8 : kDecThreads, (kF8 && kR > 16) ? 1 : 2)
     sink_attn_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                             const __grid_constant__ CUtensorMap tm_v, const DecParams p) {
+  constexpr int kStages = kF8 ? kDecStages8 : kDecStages;
+  constexpr int kTileB = kF8 ? kDecKv8Bytes : kDecKvBytes;  // bytes of one staged K or V tile
+  constexpr int kThreads = kF8 ? kDecThreads8 : kDecThreads;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   uint8_t* sK = smem;                                   // stages of K tiles
-  uint8_t* sV = sK + kDecStages * kDecKvBytes;          // stages of V tiles
-  uint8_t* sOnes = sV + kDecStages * kDecKvBytes;       // [128][64] bf16 ones
+  uint8_t* sV = sK + kStages * kTileB;                  // stages of V tiles
+  uint8_t* sVb = sV + kStages * kTileB;                 // e4m3 cache: the widened V tile (bf16)
+  uint8_t* sOnes = sVb + (kF8 ? kDecKvBytes : 0);       // [128][64] bf16 ones
   uint8_t* sP = sOnes + kDecKvBytes;                    // P^T
   uint8_t* sQ = sP + kDecPBytes;                        // Q rows (8 KB, 1024-aligned)
   DecCtl* ctl = reinterpret_cast<DecCtl*>(sQ + kDecQBytes);
@@ -206,15 +277,18 @@ __global__ void __launch_bounds__(kDecThreads, 2)
 
   if (threadIdx.x == 0) {
     mbar_init(&ctl->q_full, 1);
-    for (int s = 0; s < kDecStages; ++s) {
+    mbar_init(&ctl->q_conv, kDecTile);
+    mbar_init(&ctl->v_ready, kDecTile);
+    for (int s = 0; s < kStages; ++s) {
       mbar_init(&ctl->k_full[s], 1);
-      mbar_init(&ctl->k_empty[s], 1);
+      mbar_init(&ctl->k_empty[s], kF8 ? kDecTile : 1);  // e4m3: freed by the 128 widening threads
       mbar_init(&ctl->v_full[s], 1);
-      mbar_init(&ctl->v_empty[s], 1);
+      mbar_init(&ctl->v_empty[s], kF8 ? kDecTile : 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&ctl->s_full[b], 1);
       mbar_init(&ctl->s_free[b], kDecTile);
+      mbar_init(&ctl->kt_full[b], kDecTile);
     }
     mbar_init(&ctl->p_full, kDecTile);
     mbar_init(&ctl->pv_done, 1);
@@ -233,13 +307,14 @@ __global__ void __launch_bounds__(kDecThreads, 2)
   // Constant operands written by the threads: the ones tile, zeroed P^T and
   // zeroed Q padding rows (the TMA fills rows [0, R)).
   {
-    const uint4 ones = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
+    const uint32_t one2 = kF8 ? 0x3C003C00u : 0x3F803F80u;  // 1.0 in fp16 / bf16 pairs
+    const uint4 ones = make_uint4(one2, one2, one2, one2);
     const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
-    for (int i = threadIdx.x; i < kDecKvBytes / 16; i += kDecThreads) {
+    for (int i = threadIdx.x; i < kDecKvBytes / 16; i += kThreads) {
       reinterpret_cast<uint4*>(sOnes)[i] = ones;
       reinterpret_cast<uint4*>(sP)[i] = zero;
     }
-    for (int i = p.R * 8 + threadIdx.x; i < kDecQBytes / 16; i += kDecThreads) reinterpret_cast<uint4*>(sQ)[i] = zero;
+    for (int i = p.R * 8 + threadIdx.x; i < kDecQBytes / 16; i += kThreads) reinterpret_cast<uint4*>(sQ)[i] = zero;
     fence_proxy_async_smem();
   }
   if (warp == kDecMmaWarp) {
@@ -261,16 +336,16 @@ __global__ void __launch_bounds__(kDecThreads, 2)
       tma_load_3d(sQ, &tm_q, &ctl->q_full, 0, w.g * p.G, w.b * p.Lq);
       const int row0 = w.b * p.C + w.z0;
       for (int i = 0; i < w.n; ++i) {
-        const int s = i % kDecStages;
-        const uint32_t par = ((i / kDecStages) - 1) & 1;
-        if (i >= kDecStages && !mbar_wait(&ctl->k_empty[s], par, abort, &g_device_error, kDevErrTimeoutProducer))
+        const int s = i % kStages;
+        const uint32_t par = ((i / kStages) - 1) & 1;
+        if (i >= kStages && !mbar_wait(&ctl->k_empty[s], par, abort, &g_device_error, kDevErrTimeoutProducer))
           break;
-        mbar_arrive_expect_tx(&ctl->k_full[s], kDecKvBytes);
-        tma_load_3d(sK + s * kDecKvBytes, &tm_k, &ctl->k_full[s], 0, w.g, row0 + i * kDecTile);
-        if (i >= kDecStages && !mbar_wait(&ctl->v_empty[s], par, abort, &g_device_error, kDevErrTimeoutProducer))
+        mbar_arrive_expect_tx(&ctl->k_full[s], kTileB);
+        tma_load_3d(sK + s * kTileB, &tm_k, &ctl->k_full[s], 0, w.g, row0 + i * kDecTile);
+        if (i >= kStages && !mbar_wait(&ctl->v_empty[s], par, abort, &g_device_error, kDevErrTimeoutProducer))
           break;
-        mbar_arrive_expect_tx(&ctl->v_full[s], kDecKvBytes);
-        tma_load_3d(sV + s * kDecKvBytes, &tm_v, &ctl->v_full[s], 0, w.g, row0 + i * kDecTile);
+        mbar_arrive_expect_tx(&ctl->v_full[s], kTileB);
+        tma_load_3d(sV + s * kTileB, &tm_v, &ctl->v_full[s], 0, w.g, row0 + i * kDecTile);
       }
     }
   } else if (warp == kDecMmaWarp) {
@@ -283,41 +358,117 @@ __global__ void __launch_bounds__(kDecThreads, 2)
       const uint32_t q_addr = smem_u32(sQ);
       const uint32_t ones_addr = smem_u32(sOnes);
       const uint32_t p_addr = smem_u32(sP);
-      bool ok = mbar_wait(&ctl->q_full, 0, abort, &g_device_error, kDevErrTimeoutMma);
+      bool ok = kF8 ? mbar_wait(&ctl->q_conv, 0, abort, &g_device_error, kDevErrTimeoutMma)
+                    : mbar_wait(&ctl->q_full, 0, abort, &g_device_error, kDevErrTimeoutMma);
       for (int i = 0; ok && i <= w.n; ++i) {
         if (i < w.n) {
           const int b = i & 1;
-          const int s = i % kDecStages;
+          const int s = i % kStages;
+          // e4m3: K_i widened into TMEM buffer b by the softmax threads.
           ok = (i < 2 || mbar_wait(&ctl->s_free[b], ((i >> 1) - 1) & 1, abort, &g_device_error, kDevErrTimeoutMma)) &&
-               mbar_wait(&ctl->k_full[s], (i / kDecStages) & 1, abort, &g_device_error, kDevErrTimeoutMma);
+               (kF8 ? mbar_wait(&ctl->kt_full[b], (i >> 1) & 1, abort, &g_device_error, kDevErrTimeoutMma)
+                    : mbar_wait(&ctl->k_full[s], (i / kStages) & 1, abort, &g_device_error, kDevErrTimeoutMma));
           if (!ok) break;
           tc_fence_after();
-          dec_issue_qk(tS + b * kDecRows, smem_u32(sK + s * kDecKvBytes), q_addr);
-          tc_commit(&ctl->s_full[b]);
-          tc_commit(&ctl->k_empty[s]);
+          if constexpr (kF8) {
+            dec_issue_qk_ts(tS + b * kDecRows, tmem + kDecTmemK + 32 * b, q_addr);
+            tc_commit(&ctl->s_full[b]);
+          } else {
+            dec_issue_qk(tS + b * kDecRows, smem_u32(sK + s * kDecKvBytes), q_addr);
+            tc_commit(&ctl->s_full[b]);
+            tc_commit(&ctl->k_empty[s]);
+          }
         }
         if (i >= 1) {
           const int j = i - 1;
-          const int s = j % kDecStages;
+          const int s = j % kStages;
+          // e4m3: V_j widened into the fp16 tile (v_ready).
           ok = mbar_wait(&ctl->p_full, j & 1, abort, &g_device_error, kDevErrTimeoutMma) &&
-               mbar_wait(&ctl->v_full[s], (j / kDecStages) & 1, abort, &g_device_error, kDevErrTimeoutMma);
+               (kF8 ? mbar_wait(&ctl->v_ready, j & 1, abort, &g_device_error, kDevErrTimeoutMma)
+                    : mbar_wait(&ctl->v_full[s], (j / kStages) & 1, abort, &g_device_error, kDevErrTimeoutMma));
           if (!ok) break;
           tc_fence_after();
-          dec_issue_pv(tO, smem_u32(sV + s * kDecKvBytes), ones_addr, p_addr, j > 0);
+          dec_issue_pv<kF8>(tO, kF8 ? smem_u32(sVb) : smem_u32(sV + s * kDecKvBytes), ones_addr, p_addr, j > 0);
           tc_commit(&ctl->pv_done);
-          tc_commit(&ctl->v_empty[s]);
+          if constexpr (!kF8) tc_commit(&ctl->v_empty[s]);
         }
       }
       if (ok) tc_commit(&ctl->o_full);
+    }
+  } else if (warp >= kDecConvWarp0) {
+    // ------------------- e4m3 cache: widen K and V, one slot per thread
+    if constexpr (kF8) {
+      const int kl = 32 * (warp & 3) + (threadIdx.x & 31);  // slot == the TMEM lane this warp may access
+      const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+      bool ok = true;
+      if (w.n > 0) {
+        // Q (bf16, as loaded) -> fp16 in place: elementwise, so the swizzle
+        // does not matter; the zeroed padding rows stay zero.
+        ok = mbar_wait(&ctl->q_full, 0, abort, &g_device_error, kDevErrTimeoutDecode);
+        if (ok) {
+          uint32_t* qw = reinterpret_cast<uint32_t*>(sQ);
+          for (int e = kl; e < kDecQBytes / 4; e += kDecTile) qw[e] = bf16x2_to_f16x2_sat(qw[e]);
+          fence_proxy_async_smem();
+          mbar_arrive(&ctl->q_conv);
+        }
+      }
+      for (int i = 0; ok && i < w.n; ++i) {
+        const int b = i & 1;
+        const int s = i % kStages;
+        uint32_t buf[32];
+        // K_i -> TMEM buffer b, whose last reader was the S^T MMA of tile i-2.
+        if (i >= 2) {
+          ok = mbar_wait(&ctl->s_full[b], ((i - 2) >> 1) & 1, abort, &g_device_error, kDevErrTimeoutDecode);
+          if (!ok) break;
+          tc_fence_after();
+        }
+        ok = mbar_wait(&ctl->k_full[s], (i / kStages) & 1, abort, &g_device_error, kDevErrTimeoutDecode);
+        if (!ok) break;
+        dec_row_e4m3_to_f16(sK + s * kTileB + kl * kHeadDim, buf);
+        tmem_st32(tmem + lane_base + kDecTmemK + 32 * b, buf);
+        // Release the byte stage only after its values have been consumed
+        // (a shared load may still be in flight until its result is used),
+        // and order these generic reads before the next TMA write there.
+        fence_proxy_async_smem();
+        mbar_arrive(&ctl->k_empty[s]);
+        tc_fence_before();
+        mbar_arrive(&ctl->kt_full[b]);
+        // V_i -> the fp16 tile, whose last reader was the PV MMA of tile i-1.
+        // A slot that holds no token may hold any bits (NaN included) and
+        // its V row is still multiplied by P = 0: it becomes zeros.
+        if (i >= 1) {
+          ok = mbar_wait(&ctl->pv_done, (i - 1) & 1, abort, &g_device_error, kDevErrTimeoutDecode);
+          if (!ok) break;
+        }
+        ok = mbar_wait(&ctl->v_full[s], (i / kStages) & 1, abort, &g_device_error, kDevErrTimeoutDecode);
+        if (!ok) break;
+        const int z = w.z0 + i * kDecTile + kl;
+        const int pos = z < p.C ? dec_slot_pos(z, w.L, p.C) : -1;
+        if (pos >= 0) {
+          dec_row_e4m3_to_f16(sV + s * kTileB + kl * kHeadDim, buf);
+        } else {
+#pragma unroll
+          for (int c = 0; c < 32; ++c) buf[c] = 0u;
+        }
+        uint8_t* vline = sVb + (kl >> 3) * 1024 + (kl & 7) * 128;
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          *reinterpret_cast<uint4*>(vline + ((c ^ (kl & 7)) << 4)) =
+              make_uint4(buf[4 * c], buf[4 * c + 1], buf[4 * c + 2], buf[4 * c + 3]);
+        fence_proxy_async_smem();  // the fp16 tile for the MMA; the byte reads before the next TMA
+        mbar_arrive(&ctl->v_empty[s]);
+        mbar_arrive(&ctl->v_ready);
+      }
     }
   } else {
     // ---------------------------------------- softmax (1 key per thread)
     const int kl = threadIdx.x;  // slot within the tile == TMEM lane
     const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-    const float sl2 = p.scale_log2;
+    // e4m3: logits carry k_scale, O carries v_scale.
+    const float sl2 = kF8 ? p.scale_log2 * __ldg(p.k_scale + w.g) : p.scale_log2;
     uint32_t sync_phase = 0;
     bool ok = true;
-    for (int i = 0; i < w.n; ++i) {
+    for (int i = 0; ok && i < w.n; ++i) {
       const int b = i & 1;
       ok = mbar_wait(&ctl->s_full[b], (i >> 1) & 1, abort, &g_device_error, kDevErrTimeoutDecode);
       if (!ok) break;
@@ -378,7 +529,7 @@ __global__ void __launch_bounds__(kDecThreads, 2)
         const float m0 = ctl->m_ref[2 * c], m1 = ctl->m_ref[2 * c + 1];
         const float e0 = ex2_approx(x[2 * c] - (m0 == -INFINITY ? 0.f : m0));
         const float e1 = ex2_approx(x[2 * c + 1] - (m1 == -INFINITY ? 0.f : m1));
-        pk[c] = pack_bf16x2(e0, e1);
+        pk[c] = kF8 ? pack_f16x2(e0, e1) : pack_bf16x2(e0, e1);
       }
       // The previous PV read P^T and wrote O^T: wait for it before both.
       if (i > 0) {
@@ -397,10 +548,10 @@ __global__ void __launch_bounds__(kDecThreads, 2)
       }
       // A slot that holds no token (never written, or past this sequence's
       // C slots) may hold any bits, NaN included, and its V row is still
-      // multiplied by P = 0: zero that row of the staged V tile.
-      if (pos < 0) {
-        const int sv = i % kDecStages;
-        ok = mbar_wait(&ctl->v_full[sv], (i / kDecStages) & 1, abort, &g_device_error, kDevErrTimeoutDecode);
+      // multiplied by P = 0: its row of the V operand is zeroed.
+      if (!kF8 && pos < 0) {
+        const int sv = i % kStages;
+        ok = mbar_wait(&ctl->v_full[sv], (i / kStages) & 1, abort, &g_device_error, kDevErrTimeoutDecode);
         if (!ok) break;
         uint4* vrow = reinterpret_cast<uint4*>(sV + sv * kDecKvBytes + (kl >> 3) * 1024 + (kl & 7) * 128);
 #pragma unroll
@@ -434,9 +585,10 @@ __global__ void __launch_bounds__(kDecThreads, 2)
       if (warp < 2) {
         // Lanes 0..63: head dim kl of every query row.
         float* dst = p.o_part + cta * kDecRows * kHeadDim + kl;
+        const float vs = kF8 ? __ldg(p.v_scale + w.g) : 1.f;
 #pragma unroll
         for (int n = 0; n < kR; ++n)
-          if (n < p.R) dst[n * kHeadDim] = have ? __uint_as_float(o[n]) : 0.f;
+          if (n < p.R) dst[n * kHeadDim] = have ? __uint_as_float(o[n]) * vs : 0.f;
       } else if (kl == 64) {
         // Lane 64: the row sums.
 #pragma unroll
@@ -517,6 +669,48 @@ __global__ void __launch_bounds__(256) sink_attn_cache_append_kernel(const DecPa
   const size_t dst = ((static_cast<size_t>(b) * p.C + slot) * p.Hkv + g) * kChunks + c;
   if (is_v) v_cache[dst] = v_new[e];
   else k_cache[dst] = k_new[e];
+}
+
+// Appends the new tokens to an e4m3 cache: code = e4m3(x * (1 / scale[g]))
+// (round to nearest even, saturated to the largest finite code, +-448).  One
+// thread per 16 codes (two 16-byte loads of bf16 input, one 16-byte store).
+__device__ __forceinline__ uint32_t f32x2_to_e4m3x2(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+__global__ void __launch_bounds__(256) sink_attn_cache_append_e4m3_kernel(const DecParams p, const uint4* k_new,
+                                                                          const uint4* v_new, uint4* k_cache,
+                                                                          uint4* v_cache) {
+  constexpr int kChunks = kHeadDim / 16;  // 16-code chunks per [D] row
+  const long long total = static_cast<long long>(p.batch) * p.Lq * p.Hkv * kChunks;
+  const long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= 2 * total) return;
+  const bool is_v = i >= total;
+  const long long e = is_v ? i - total : i;
+  const int c = static_cast<int>(e % kChunks);
+  const long long r = e / kChunks;  // (b * Lq + t) * Hkv + g
+  const int g = static_cast<int>(r % p.Hkv);
+  const long long bt = r / p.Hkv;
+  const int b = static_cast<int>(bt / p.Lq);
+  const int t = static_cast<int>(bt % p.Lq);
+  const int L0 = __ldg(p.seqlens + b);
+  if (L0 < 0) return;  // reported by the attention kernel
+  const int slot = (L0 + t) % p.C;
+  const float inv = 1.f / __ldg((is_v ? p.v_scale : p.k_scale) + g);
+  const uint4* src = (is_v ? v_new : k_new) + r * (kHeadDim / 8) + 2 * c;  // 16 bf16
+  uint32_t w[8];
+  const uint4 a = src[0], bq = src[1];
+  const uint32_t in[8] = {a.x, a.y, a.z, a.w, bq.x, bq.y, bq.z, bq.w};
+#pragma unroll
+  for (int u = 0; u < 8; ++u) {
+    const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&in[u]));
+    w[u] = f32x2_to_e4m3x2(f.x * inv, f.y * inv);
+  }
+  const size_t dst = ((static_cast<size_t>(b) * p.C + slot) * p.Hkv + g) * kChunks + c;
+  (is_v ? v_cache : k_cache)[dst] = make_uint4(w[0] | (w[1] << 16), w[2] | (w[3] << 16), w[4] | (w[5] << 16),
+                                               w[6] | (w[7] << 16));
 }
 
 }  // namespace sa

@@ -120,6 +120,7 @@ sink_attn_status plan_decode(const sink_attn_decode_dims* d, int window, float s
   p.scale_log2 = scale * kLog2e;
   p.seqlens = nullptr;
   p.sinks = nullptr;
+  p.k_scale = p.v_scale = nullptr;
   p.o_part = p.m_part = p.l_part = nullptr;
   // Upper bound on the 128-slot tiles one sequence scans.
   int64_t slots = std::min<int64_t>(d->cache_capacity, d->max_seqlen);
@@ -333,53 +334,99 @@ int sink_attn_decode_launches(const sink_attn_decode_dims* d) {
   return d->batch > 0 ? 3 : 0;
 }
 
-sink_attn_status sink_attn_decode(const sink_attn_decode_dims* d, const void* q, const void* k_new,
-                                  const void* v_new, void* k_cache, void* v_cache, const int* cache_seqlens,
-                                  const float* sinks, int window, float scale, void* out, float* lse,
-                                  void* workspace, size_t workspace_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+
+sink_attn_status decode_impl(const sink_attn_decode_dims* d, const void* q, const void* k_new, const void* v_new,
+                             void* k_cache, void* v_cache, const int* cache_seqlens, const float* k_scale,
+                             const float* v_scale, bool e4m3, const float* sinks, int window, float scale, void* out,
+                             float* lse, void* workspace, size_t workspace_bytes, void* stream) {
   DecPlan plan;
   sink_attn_status st = plan_decode(d, window, scale, &plan);
   if (st != SINK_ATTN_OK) return st;
   if (d->batch == 0) return SINK_ATTN_OK;
-  if (!q || !k_new || !v_new || !k_cache || !v_cache || !cache_seqlens || !sinks || !out || !lse)
+  if (!q || !k_new || !v_new || !k_cache || !v_cache || !cache_seqlens || !sinks || !out || !lse ||
+      (e4m3 && (!k_scale || !v_scale)))
     return SINK_ATTN_ERR_NULL;
   if (!aligned16(q) || !aligned16(k_new) || !aligned16(v_new) || !aligned16(k_cache) || !aligned16(v_cache) ||
       !aligned16(out) || (reinterpret_cast<uintptr_t>(lse) & 3u) || (reinterpret_cast<uintptr_t>(sinks) & 3u) ||
-      (reinterpret_cast<uintptr_t>(cache_seqlens) & 3u))
+      (reinterpret_cast<uintptr_t>(cache_seqlens) & 3u) || (reinterpret_cast<uintptr_t>(k_scale) & 3u) ||
+      (reinterpret_cast<uintptr_t>(v_scale) & 3u))
     return SINK_ATTN_ERR_ALIGN;
   if (!workspace || workspace_bytes < plan.total || (reinterpret_cast<uintptr_t>(workspace) & 255u))
     return SINK_ATTN_ERR_WORKSPACE;
   DecParams p = plan.p;
   p.seqlens = cache_seqlens;
   p.sinks = sinks;
+  p.k_scale = k_scale;
+  p.v_scale = v_scale;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   p.o_part = reinterpret_cast<float*>(ws + plan.o_off);
   p.m_part = reinterpret_cast<float*>(ws + plan.m_off);
   p.l_part = reinterpret_cast<float*>(ws + plan.l_off);
 
   CUtensorMap tq, tk, tv;
-  if (!make_map_3d(&tq, q, kHeadDim, p.Hq, p.batch * p.Lq, p.G, p.Lq) ||
-      !make_map_3d(&tk, k_cache, kHeadDim, p.Hkv, p.batch * p.C, 1, kDecTile) ||
-      !make_map_3d(&tv, v_cache, kHeadDim, p.Hkv, p.batch * p.C, 1, kDecTile))
+  if (!make_map_3d(&tq, q, kHeadDim, p.Hq, p.batch * p.Lq, p.G, p.Lq)) return SINK_ATTN_ERR_CUDA;
+  if (e4m3) {
+    if (!make_map_3d_u8(&tk, k_cache, kHeadDim, p.Hkv, p.batch * p.C, 1, kDecTile) ||
+        !make_map_3d_u8(&tv, v_cache, kHeadDim, p.Hkv, p.batch * p.C, 1, kDecTile))
+      return SINK_ATTN_ERR_CUDA;
+  } else if (!make_map_3d(&tk, k_cache, kHeadDim, p.Hkv, p.batch * p.C, 1, kDecTile) ||
+             !make_map_3d(&tv, v_cache, kHeadDim, p.Hkv, p.batch * p.C, 1, kDecTile)) {
     return SINK_ATTN_ERR_CUDA;
+  }
   // Register arrays sized for the real query rows.
-  void (*kern)(CUtensorMap, CUtensorMap, CUtensorMap, DecParams) =
-      p.R <= 16 ? sink_attn_decode_kernel<16> : (p.R <= 32 ? sink_attn_decode_kernel<32> : sink_attn_decode_kernel<64>);
-  static int smem_set[3] = {0, 0, 0};
-  if (!set_smem_once(kern, kDecSmemBytes, &smem_set[p.R <= 16 ? 0 : (p.R <= 32 ? 1 : 2)])) return SINK_ATTN_ERR_CUDA;
+  using Kern = void (*)(CUtensorMap, CUtensorMap, CUtensorMap, DecParams);
+  static const Kern kerns[2][3] = {
+      {sink_attn_decode_kernel<16, false>, sink_attn_decode_kernel<32, false>, sink_attn_decode_kernel<64, false>},
+      {sink_attn_decode_kernel<16, true>, sink_attn_decode_kernel<32, true>, sink_attn_decode_kernel<64, true>}};
+  static int smem_set[2][3] = {{0, 0, 0}, {0, 0, 0}};
+  const int vi = p.R <= 16 ? 0 : (p.R <= 32 ? 1 : 2);
+  const Kern kern = kerns[e4m3][vi];
+  const size_t smem = e4m3 ? kDecSmemBytes8 : kDecSmemBytes;
+  if (!set_smem_once(kern, smem, &smem_set[e4m3][vi])) return SINK_ATTN_ERR_CUDA;
   const long long ctas = static_cast<long long>(p.batch) * p.Hkv * p.n_split;
   if (ctas > 0x7fffffff) return SINK_ATTN_ERR_UNSUPPORTED;
 
   cudaStream_t st_ = static_cast<cudaStream_t>(stream);
-  const long long chunks = 2LL * p.batch * p.Lq * p.Hkv * (kHeadDim * 2 / 16);
-  sink_attn_cache_append_kernel<<<static_cast<unsigned>((chunks + 255) / 256), 256, 0, st_>>>(
-      p, static_cast<const uint4*>(k_new), static_cast<const uint4*>(v_new), static_cast<uint4*>(k_cache),
-      static_cast<uint4*>(v_cache));
-  kern<<<static_cast<unsigned>(ctas), kDecThreads, kDecSmemBytes, st_>>>(tq, tk, tv, p);
+  if (e4m3) {
+    const long long chunks = 2LL * p.batch * p.Lq * p.Hkv * (kHeadDim / 16);
+    sink_attn_cache_append_e4m3_kernel<<<static_cast<unsigned>((chunks + 255) / 256), 256, 0, st_>>>(
+        p, static_cast<const uint4*>(k_new), static_cast<const uint4*>(v_new), static_cast<uint4*>(k_cache),
+        static_cast<uint4*>(v_cache));
+  } else {
+    const long long chunks = 2LL * p.batch * p.Lq * p.Hkv * (kHeadDim * 2 / 16);
+    sink_attn_cache_append_kernel<<<static_cast<unsigned>((chunks + 255) / 256), 256, 0, st_>>>(
+        p, static_cast<const uint4*>(k_new), static_cast<const uint4*>(v_new), static_cast<uint4*>(k_cache),
+        static_cast<uint4*>(v_cache));
+  }
+  kern<<<static_cast<unsigned>(ctas), e4m3 ? kDecThreads8 : kDecThreads, smem, st_>>>(tq, tk, tv, p);
   const long long rows = static_cast<long long>(p.batch) * p.Lq * p.Hq;
   sink_attn_decode_combine_kernel<<<static_cast<unsigned>((rows + 3) / 4), 128, 0, st_>>>(
       p, static_cast<__nv_bfloat16*>(out), lse);
   return cudaPeekAtLastError() == cudaSuccess ? SINK_ATTN_OK : SINK_ATTN_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+sink_attn_status sink_attn_decode(const sink_attn_decode_dims* d, const void* q, const void* k_new,
+                                  const void* v_new, void* k_cache, void* v_cache, const int* cache_seqlens,
+                                  const float* sinks, int window, float scale, void* out, float* lse,
+                                  void* workspace, size_t workspace_bytes, void* stream) {
+  return decode_impl(d, q, k_new, v_new, k_cache, v_cache, cache_seqlens, nullptr, nullptr, false, sinks, window,
+                     scale, out, lse, workspace, workspace_bytes, stream);
+}
+
+sink_attn_status sink_attn_decode_e4m3(const sink_attn_decode_dims* d, const void* q, const void* k_new,
+                                       const void* v_new, void* k_cache, void* v_cache, const int* cache_seqlens,
+                                       const float* k_scale, const float* v_scale, const float* sinks, int window,
+                                       float scale, void* out, float* lse, void* workspace, size_t workspace_bytes,
+                                       void* stream) {
+  return decode_impl(d, q, k_new, v_new, k_cache, v_cache, cache_seqlens, k_scale, v_scale, true, sinks, window,
+                     scale, out, lse, workspace, workspace_bytes, stream);
 }
 
 }  // extern "C"

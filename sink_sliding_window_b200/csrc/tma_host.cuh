@@ -60,4 +60,22 @@ inline bool make_map_3d_f32(CUtensorMap* map, const void* base, int inner, int m
   return r == CUDA_SUCCESS;
 }
 
+// 3-D byte view [outer][mid][inner] (e.g. an e4m3 cache), no swizzle: a box
+// lands in shared memory as plain rows of `inner` bytes.
+inline bool make_map_3d_u8(CUtensorMap* map, const void* base, int inner, int mid, int outer, int box_mid,
+                           int box_outer) {
+  EncodeTiledFn enc = get_encode_tiled();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(mid),
+                        static_cast<cuuint64_t>(outer)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(inner) * mid};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(inner), static_cast<cuuint32_t>(box_mid),
+                       static_cast<cuuint32_t>(box_outer)};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 }  // namespace sa

@@ -27,7 +27,8 @@ STATUS = {
 
 EXPORTS = ("sink_attn_fwd", "sink_attn_bwd", "sink_attn_bwd_workspace_size", "sink_attn_status_string",
            "sink_attn_device_error", "sink_attn_fwd_launches", "sink_attn_bwd_launches", "sink_attn_profile_events",
-           "sink_attn_decode", "sink_attn_decode_workspace_size", "sink_attn_decode_launches")
+           "sink_attn_decode", "sink_attn_decode_workspace_size", "sink_attn_decode_launches",
+           "sink_attn_decode_e4m3")
 
 
 class SinkAttnError(RuntimeError):
@@ -81,6 +82,9 @@ def load():
         DD = ctypes.POINTER(DecodeDims)
         L.sink_attn_decode.argtypes = [DD, P, P, P, P, P, P, P, I, ctypes.c_float, P, P, P, ctypes.c_size_t, P]
         L.sink_attn_decode.restype = I
+        L.sink_attn_decode_e4m3.argtypes = [DD, P, P, P, P, P, P, P, P, P, I, ctypes.c_float, P, P, P,
+                                            ctypes.c_size_t, P]
+        L.sink_attn_decode_e4m3.restype = I
         L.sink_attn_decode_workspace_size.argtypes = [DD, I]
         L.sink_attn_decode_workspace_size.restype = ctypes.c_size_t
         L.sink_attn_decode_launches.argtypes = [DD]
@@ -212,6 +216,35 @@ def decode(q, k_new, v_new, k_cache, v_cache, cache_seqlens, sinks, window=0, sc
                             _ptr(workspace), ctypes.c_size_t(workspace.numel()), _stream_handle(stream))
     if st != 0:
         raise SinkAttnError(st, "sink_attn_decode")
+    return out, lse
+
+
+def decode_e4m3(q, k_new, v_new, k_cache, v_cache, cache_seqlens, k_scale, v_scale, sinks, window=0, scale=None, *,
+                max_seqlen=None, out=None, lse=None, workspace=None, stream=None):
+    """sink_attn_decode_e4m3: as decode(), with k_cache / v_cache holding e4m3
+    codes ([B, C, Hkv, D] uint8 or torch.float8_e4m3fn) and k_scale / v_scale
+    fp32 [Hkv] dequantisation scales."""
+    B, Lq, Hq, D = q.shape
+    C, Hkv = k_cache.shape[1], k_cache.shape[2]
+    if max_seqlen is None:
+        max_seqlen = C + Lq
+    if scale is None:
+        scale = D ** -0.5
+    dims = decode_dims(B, Lq, C, max_seqlen, Hq, Hkv, D)
+    L = load()
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((Hq, B * Lq), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        need = int(L.sink_attn_decode_workspace_size(ctypes.byref(dims), int(window)))
+        workspace = torch.empty((max(need, 1),), dtype=torch.uint8, device=q.device)
+    st = L.sink_attn_decode_e4m3(ctypes.byref(dims), _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_cache),
+                                 _ptr(v_cache), _ptr(cache_seqlens), _ptr(k_scale), _ptr(v_scale), _ptr(sinks),
+                                 int(window), float(scale), _ptr(out), _ptr(lse), _ptr(workspace),
+                                 ctypes.c_size_t(workspace.numel()), _stream_handle(stream))
+    if st != 0:
+        raise SinkAttnError(st, "sink_attn_decode_e4m3")
     return out, lse
 
 

@@ -150,3 +150,77 @@ def test_gpt_oss_decode_full_size(ops, window, C):
 def test_launch_count(ops):
     assert ops.decode_launches(4, 1, 256, 257, 64, 8) == 3
     assert ops.decode_launches(0, 1, 256, 257, 64, 8) == 0
+
+
+# ----------------------------------------------------------------- e4m3 cache
+def _run_e4m3(ops, cached, Lq, Hq, Hkv, C, window, seed, seqs=None):
+    """The e4m3-cache decode: history tokens enter the cache as host-quantised
+    codes (per-head scale = amax / 448), the new tokens are quantised by the
+    call.  The oracle gets the dequantised values code * scale exactly (fp64),
+    so the comparison measures the kernel, not the quantisation."""
+    import torch
+    from tests import e4m3
+    a = synth.decode_inputs(seed, cached, Lq, Hq, Hkv)
+    cu = a["cu"]
+    B = len(cached)
+    kf = synth.bf16_bits_to_f32(a["k"])
+    vf = synth.bf16_bits_to_f32(a["v"])
+    ks = (np.abs(kf).max(axis=(0, 2)) / np.float32(448.0)).astype(np.float32)
+    vs = (np.abs(vf).max(axis=(0, 2)) / np.float32(448.0)).astype(np.float32)
+    ck = e4m3.quantize(kf * (np.float32(1.0) / ks)[None, :, None])
+    cv = e4m3.quantize(vf * (np.float32(1.0) / vs)[None, :, None])
+    kc0 = np.full((B, C, Hkv, 64), 0x7F, np.uint8)  # unused slots hold the NaN code
+    vc0 = np.full((B, C, Hkv, 64), 0x7F, np.uint8)
+    for b in range(B):
+        for p in range(int(cached[b])):
+            kc0[b, p % C] = ck[int(cu[b]) + p]
+            vc0[b, p % C] = cv[int(cu[b]) + p]
+    new_idx = np.concatenate([np.arange(int(cu[b]) + int(cached[b]), int(cu[b + 1])) for b in range(B)])
+    k_new = a["k"][new_idx].reshape(B, Lq, Hkv, 64)
+    v_new = a["v"][new_idx].reshape(B, Lq, Hkv, 64)
+    kc, vc = torch.from_numpy(kc0).cuda(), torch.from_numpy(vc0).cuda()
+    out, lse = ops.decode_e4m3(dev_bf16(a["q_new"]), dev_bf16(k_new), dev_bf16(v_new), kc, vc,
+                               dev(np.asarray(cached, np.int32)), dev(ks), dev(vs), dev(a["sinks"]), window, SCALE,
+                               max_seqlen=int(max(cached)) + Lq)
+    torch.cuda.synchronize()
+    assert ops.device_error() == 0
+    ke, ve = kc0.copy(), vc0.copy()
+    for b in range(B):
+        for t in range(Lq):
+            ke[b, (int(cached[b]) + t) % C] = ck[int(cu[b]) + int(cached[b]) + t]
+            ve[b, (int(cached[b]) + t) % C] = cv[int(cu[b]) + int(cached[b]) + t]
+    assert np.array_equal(kc.cpu().numpy(), ke), "e4m3 k cache after append (quantisation of the new tokens)"
+    assert np.array_equal(vc.cpu().numpy(), ve), "e4m3 v cache after append"
+    kd = e4m3.decode(ck) * ks[None, :, None].astype(np.float64)
+    vd = e4m3.decode(cv) * vs[None, :, None].astype(np.float64)
+    qd = synth.bf16_bits_to_f32(a["q_new"]).astype(np.float64)
+    seqs = list(range(B)) if seqs is None else list(seqs)
+    outs, lses = [], []
+    for b in seqs:
+        lo, hi = int(cu[b]), int(cu[b + 1])
+        L = hi - lo
+        q = np.zeros((L, Hq, 64))
+        q[int(cached[b]):] = qd[b]
+        rows = np.arange(int(cached[b]), L, dtype=np.int64)
+        o, l = oracle.fwd_rows(q, kd[lo:hi], vd[lo:hi], a["sinks"].astype(np.float64), np.array([0, L], np.int32),
+                               window, SCALE, rows)
+        outs.append(o)
+        lses.append(l)
+    got_o = host_f64(out)[seqs].reshape(-1, Hq, 64)
+    got_l = host_f64(lse).reshape(Hq, B, Lq)[:, seqs].reshape(Hq, -1)
+    check(got_o, np.concatenate(outs), TOL_OUT, "e4m3 decode out")
+    check(got_l, np.concatenate(lses, axis=1), TOL_LSE, "e4m3 decode lse")
+
+
+@pytest.mark.parametrize("window,C,Lq", [(0, 1152, 1), (100, 1152, 1), (128, 128, 1), (128, 129, 2), (16, 18, 3)])
+def test_e4m3_cache(ops, window, C, Lq):
+    _run_e4m3(ops, [0, 1, 99, 127, 128, 129, 300, 1000], Lq, 16, 2, C, window, seed=60 + Lq)
+
+
+@pytest.mark.parametrize("G,Lq", [(8, 4), (16, 4)])
+def test_e4m3_cache_row_variants(ops, G, Lq):
+    _run_e4m3(ops, [0, 64, 257], Lq, 2 * G, 2, 512, 0, seed=70 + G)
+
+
+def test_e4m3_cache_gpt_oss_full_size(ops):
+    _run_e4m3(ops, [8191] * 62 + [0, 4000], 1, 64, 8, 8192, 0, seed=80, seqs=[0, 31, 62, 63])
