@@ -6,9 +6,9 @@
 //   dv_j = sum_{i,h in group} P_ij dout_i,  dsinks_h = -sum_i P_sink,i D_i
 //
 // Three launches on the caller's stream:
-//   1. bwd_preprocess: D_i; lse_i*log2(e) and D_i re-laid out in query-tile
-//      row order (so the main kernel fetches a tile's 128 values with one bulk
-//      copy); the first allowed key of every token; per-block partial sums of
+//   1. bwd_preprocess: D_i; -lse_i*log2(e) and -D_i re-laid out in
+//      query-tile row order (so the main kernel fetches a tile's 128 values
+//      with one bulk copy); the first allowed key of every token; per-block partial sums of
 //      -P_sink,i D_i (fixed order); and zeroes the fp32 dq accumulator.
 //   2. bwd_main (tcgen05): one CTA per 128-key tile of one key/value head g,
 //      visiting every query tile (the forward's 128 rows = 128/G tokens x G
@@ -37,8 +37,8 @@ constexpr int kFinishThreads = 256;
 struct BwdWorkspace {
   size_t dq_acc;    // fp32 [T][Hq][D]
   size_t Dvec;      // fp32 [Hq][T]
-  size_t lse2_blk;  // fp32 [num_qblocks][Hkv][128]  lse*log2(e) in tile-row order (+inf for padding rows)
-  size_t D_blk;     // fp32 [num_qblocks][Hkv][128]  D in tile-row order (0 for padding rows)
+  size_t lse2_blk;  // fp32 [num_qblocks][Hkv][128]  -lse*log2(e) in tile-row order (-inf for padding rows)
+  size_t D_blk;     // fp32 [num_qblocks][Hkv][128]  -D in tile-row order (0 for padding rows)
   size_t lo_blk;    // int  [num_qblocks][128]       first allowed key per token of the tile
   size_t partials;  // fp32 [Hq][num_pre_blocks]
   int num_pre_blocks;
@@ -137,15 +137,16 @@ __global__ void __launch_bounds__(kPreThreads) sink_attn_bwd_preprocess_kernel(c
       if (t < geo.T) {
         const float lse = __ldg(p.lse + static_cast<size_t>(h) * geo.T + t);
         p.Dvec[static_cast<size_t>(h) * geo.T + t] = D;
-        p.D_blk[bi] = D;
-        p.lse2_blk[bi] = lse * kLog2e;
+        // Stored negated: the main kernel adds them with two-wide fp32 ops.
+        p.D_blk[bi] = -D;
+        p.lse2_blk[bi] = -(lse * kLog2e);
         const float psink = ex2_approx((__ldg(p.sinks + h) - lse) * kLog2e);  // e^{s_h - lse}; 0 for s = -inf
         contrib -= psink * D;
         if (h == 0) p.lo_blk[static_cast<size_t>(qb) * kBlockM + pos] = first_key(geo, t);
       } else {
         // padding rows of the last query tile: P = 0 and dS = 0 there
         p.D_blk[bi] = 0.f;
-        p.lse2_blk[bi] = INFINITY;
+        p.lse2_blk[bi] = -INFINITY;
         if (h == 0) p.lo_blk[static_cast<size_t>(qb) * kBlockM + pos] = 0x7fffffff;
       }
     }
@@ -215,8 +216,9 @@ constexpr int kBwdWarpProducer = 8;
 constexpr int kBwdWarpMma = 9;
 constexpr int kBwdWarpDq0 = 10;     // warps 10..13
 constexpr uint32_t kBwdTmemCols = 512;
-constexpr uint32_t kBwdTmemS0 = 0;    // S^T buffer 0: fp32 [128 keys][128 rows]; P^T bf16 in cols 0..63,
-constexpr uint32_t kBwdTmemS1 = 128;  //   the tile's dQ (fp32 [128 rows][64]) later in cols 64..127
+constexpr uint32_t kBwdTmemS0 = 0;    // S^T buffer 0: fp32 [128 keys][128 rows]; P^T bf16 in cols 0..31
+constexpr uint32_t kBwdTmemS1 = 128;  //   (rows 0-63) and 64..95 (rows 64-127); the tile's dQ (fp32
+                                      //   [128 rows][64]) later in cols 64..127, after the dV MMA read P^T
 constexpr uint32_t kBwdTmemDP = 256;  // dP^T fp32; dS^T bf16 in cols 0..31 (rows 0-63) and 64..95 (rows 64-127)
 constexpr uint32_t kBwdTmemDV = 384;  // dV accumulator fp32 [128 keys][64]
 constexpr uint32_t kBwdTmemDK = 448;  // dK accumulator
@@ -233,8 +235,8 @@ struct BwdParams {
 };
 
 struct BwdAux {
-  float lse2[kBlockM];  // lse*log2(e) per row of the query tile
-  float D[kBlockM];
+  float lse2[kBlockM];  // -lse*log2(e) per row of the query tile (-inf for padding rows)
+  float D[kBlockM];     // -D per row
   int lo[kBlockM];      // first allowed key per token of the tile (first 128/G entries)
 };
 
@@ -248,7 +250,6 @@ struct BwdCtl {
   uint64_t dq_full;
   uint64_t dq_empty;
   uint64_t kd_full;
-  uint64_t pair_sync[4];  // the two softmax warps of one TMEM lane group (64 threads)
   uint64_t dq_sync;       // the four dQ warps (128 threads)
   uint32_t tmem_base;
   int abort;
@@ -316,10 +317,12 @@ __device__ __forceinline__ uint32_t ds_smem_offset(int key, int chunk16) {
 
 // P^T for this thread's key over the 64 query rows [64*ch, 64*ch+64) of a
 // tile: P = 2^(S^T * scale*log2e - lse2), zero where the pair is masked,
-// rounded to bf16 and packed in row pairs (pk[r/2] holds rows r, r+1).
+// rounded to bf16 and packed in row pairs (pk[r/2] holds rows r, r+1).  The
+// scaling runs two rows per instruction (a.lse2 holds -lse2).
 template <bool kMask>
 __device__ __forceinline__ void bwd_p_rows(uint32_t tS, const BwdAux& a, int ch, float sl2, int j, int q0, int G_log2,
                                            uint32_t* pk) {
+  const uint64_t sl2x2 = f32x2_pack(sl2, sl2);
 #pragma unroll
   for (int half = 0; half < 2; ++half) {
     uint32_t sr[32];
@@ -329,11 +332,15 @@ __device__ __forceinline__ void bwd_p_rows(uint32_t tS, const BwdAux& a, int ch,
     for (int c = 0; c < 32; c += 4) {
       const int col = 64 * ch + 32 * half + c;
       const float4 l4 = *reinterpret_cast<const float4*>(&a.lse2[col]);
-      const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+      float y[4];
+      f32x2_unpack(fma_f32x2(f32x2_pack(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), sl2x2,
+                             f32x2_pack(l4.x, l4.y)), y[0], y[1]);
+      f32x2_unpack(fma_f32x2(f32x2_pack(__uint_as_float(sr[c + 2]), __uint_as_float(sr[c + 3])), sl2x2,
+                             f32x2_pack(l4.z, l4.w)), y[2], y[3]);
       float pe[4];
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
-        pe[u] = ex2_approx(fmaf(__uint_as_float(sr[c + u]), sl2, -lv[u]));
+        pe[u] = ex2_approx(y[u]);
         if (kMask) {
           const int pos = (col + u) >> G_log2;
           if (!(j >= a.lo[pos] && j <= q0 + pos)) pe[u] = 0.f;
@@ -377,7 +384,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     mbar_init(&ctl->dq_full, 1);
     mbar_init(&ctl->dq_empty, 128);
     mbar_init(&ctl->kd_full, 1);
-    for (int l = 0; l < 4; ++l) mbar_init(&ctl->pair_sync[l], 64);
     mbar_init(&ctl->dq_sync, 128);
     ctl->abort = 0;
     fence_mbar_init();
@@ -471,12 +477,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tc_fence_after();
         const uint32_t q_addr = smem_u32(sQ + st * kTileBytes), do_addr = smem_u32(sDO + st * kTileBytes);
         // dV += P^T dO and dK += dS^T Q over the tile's 128 query rows.  P^T
-        // sits in cols 0..63 of the S^T buffer; dS^T in cols 0..31 (rows
-        // 0-63) and 64..95 (rows 64-127) of the dP^T region.
+        // sits in cols 0..31 (rows 0-63) and 64..95 (rows 64-127) of the S^T
+        // buffer; dS^T at the same columns of the dP^T region.
 #pragma unroll
         for (int kk = 0; kk < kBlockM / 16; ++kk) {
           const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
-          mma_ts(tDV, tSb + kk * 8, make_sdesc_sw128(do_addr + kk * 2048, kTileBytes, 1024), idesc_acc, acc);
+          mma_ts(tDV, tSb + (kk < 4 ? kk * 8 : 64 + (kk - 4) * 8),
+                 make_sdesc_sw128(do_addr + kk * 2048, kTileBytes, 1024), idesc_acc, acc);
           mma_ts(tDK, tDP + (kk < 4 ? kk * 8 : 64 + (kk - 4) * 8),
                  make_sdesc_sw128(q_addr + kk * 2048, kTileBytes, 1024), idesc_acc, acc);
         }
@@ -514,7 +521,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const int j = w.k0 + kl;                 // this thread's key
     const uint32_t lane_base = static_cast<uint32_t>(32 * lg) << 16;
     const float sl2 = p.scale_log2;
-    uint32_t pair_phase = 0;
     bool ok = true;
     for (int i = 0; i < w.nq; ++i) {
       const int st = i % kBwdStages;
@@ -537,14 +543,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         bwd_p_rows<false>(tS, a, ch, sl2, j, q0, geo.G_log2, pk);
       else
         bwd_p_rows<true>(tS, a, ch, sl2, j, q0, geo.G_log2, pk);
-      // Both warps of this lane group have read S^T: P^T (bf16) may now
-      // overwrite its first 64 columns.
-      tc_fence_before();
-      ok = group_sync(&ctl->pair_sync[lg], pair_phase, abort, kDevErrTimeoutSoftmax);
-      if (!ok) break;
-      tc_fence_after();
+      // P^T (bf16) of this warp's 64 rows over the first half of its own
+      // S^T columns (rows 0-63 -> columns 0..31, rows 64-127 -> 64..95):
+      // this warp has read them and no other warp reads them.
       __syncwarp();
-      tmem_st32_nowait(tmem + lane_base + sbuf + 32 * ch, pk);
+      tmem_st32_nowait(tmem + lane_base + sbuf + 64 * ch, pk);
       ok = mbar_wait(&ctl->dp_full, i & 1, abort, &g_device_error, kDevErrTimeoutSoftmax);
       if (!ok) break;
       tc_fence_after();
@@ -560,15 +563,19 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
         for (int c = 0; c < 32; c += 4) {
           const int col = 64 * ch + 32 * half + c;
-          const float4 d4 = *reinterpret_cast<const float4*>(&a.D[col]);
-          const float2 p01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&pk[16 * half + c / 2]));
-          const float2 p23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&pk[16 * half + c / 2 + 1]));
-          const float ds0 = p01.x * (__uint_as_float(dr[c + 0]) - d4.x);
-          const float ds1 = p01.y * (__uint_as_float(dr[c + 1]) - d4.y);
-          const float ds2 = p23.x * (__uint_as_float(dr[c + 2]) - d4.z);
-          const float ds3 = p23.y * (__uint_as_float(dr[c + 3]) - d4.w);
-          dk[c / 2] = pack_bf16x2(ds0, ds1);
-          dk[c / 2 + 1] = pack_bf16x2(ds2, ds3);
+          const float4 nd4 = *reinterpret_cast<const float4*>(&a.D[col]);  // -D
+          // dS = P (dP - D), two rows per instruction.
+          float ds[4];
+          f32x2_unpack(mul_f32x2(bf16x2_to_f32x2(pk[16 * half + c / 2]),
+                                 add_f32x2(f32x2_pack(__uint_as_float(dr[c]), __uint_as_float(dr[c + 1])),
+                                           f32x2_pack(nd4.x, nd4.y))),
+                       ds[0], ds[1]);
+          f32x2_unpack(mul_f32x2(bf16x2_to_f32x2(pk[16 * half + c / 2 + 1]),
+                                 add_f32x2(f32x2_pack(__uint_as_float(dr[c + 2]), __uint_as_float(dr[c + 3])),
+                                           f32x2_pack(nd4.z, nd4.w))),
+                       ds[2], ds[3]);
+          dk[c / 2] = pack_bf16x2(ds[0], ds[1]);
+          dk[c / 2 + 1] = pack_bf16x2(ds[2], ds[3]);
         }
         // dS^T for this warp's rows -> the first 32 columns of its own dP^T
         // column range (this warp has finished reading them).
