@@ -55,7 +55,7 @@ constexpr int kDecMmaWarp = 5;
 constexpr int kDecRows = 64;      // MMA N: query rows per CTA (G x Lq <= 64)
 constexpr int kDecTile = 128;     // slots per key tile (MMA M)
 constexpr int kDecStages = 2;      // bf16 cache: K/V tile stages
-constexpr int kDecStages8 = 3;     // e4m3 cache: byte-tile stages
+constexpr int kDecStages8 = 2;     // e4m3 cache: byte-tile stages
 constexpr int kDecQBytes = kDecRows * kHeadDim * 2;    // Q tile, [64][64] bf16
 constexpr int kDecKvBytes = kDecTile * kHeadDim * 2;   // one K or V tile, [128][64] bf16
 constexpr int kDecPBytes = kDecTile * kDecRows * 2;    // P^T tile, [128 keys][64 rows] bf16
@@ -89,11 +89,13 @@ struct DecCtl {
   uint64_t v_full[kDecStages8];
   uint64_t v_empty[kDecStages8];
   uint64_t kt_full[2];  // e4m3 cache: K of tile i widened into TMEM buffer i % 2 (128 arrivals)
-  uint64_t v_ready;     // e4m3 cache: V of tile i widened into the fp16 tile (128 arrivals)
+  uint64_t v_ready[2];  // e4m3 cache: V of tile i widened into fp16 tile i % 2, barrier i % 2
+                        // (128 arrivals; split so that a converter two tiles ahead stays unambiguous)
   uint64_t s_full[2];   // S^T of tile i in TMEM buffer i % 2
   uint64_t s_free[2];   // the softmax has loaded that S^T (128 arrivals)
   uint64_t p_full;      // P^T of tile i written (128 arrivals)
-  uint64_t pv_done;     // O^T += ... of tile i complete
+  uint64_t pv_done[2];  // O^T += ... of tile i complete, barrier i % 2 (the softmax and the e4m3
+                        // widening threads wait on different tiles' completions)
   uint64_t o_full;      // every MMA done
   uint64_t sync;        // the 128 softmax threads
   float m_ref[kDecRows];    // reference max per query row (log2 units)
@@ -106,7 +108,7 @@ struct DecCtl {
 
 constexpr size_t kDecSmemBytes = 1024 /*alignment slack*/ + kDecQBytes + 2 * kDecStages * kDecKvBytes +
                                  kDecKvBytes /*ones*/ + kDecPBytes + sizeof(DecCtl);
-constexpr size_t kDecSmemBytes8 = 1024 + kDecQBytes + 2 * kDecStages8 * kDecKv8Bytes + kDecKvBytes /*bf16 V*/ +
+constexpr size_t kDecSmemBytes8 = 1024 + kDecQBytes + 2 * kDecStages8 * kDecKv8Bytes + 2 * kDecKvBytes /*fp16 V x2*/ +
                                   kDecKvBytes /*ones*/ + kDecPBytes + sizeof(DecCtl);
 
 // Slot range of one CTA: [z0, z0 + 128 n) in 128-slot tiles.
@@ -266,8 +268,8 @@ __global__ void __launch_bounds__(kF8 ? kDecThreads8 : kDecThreads, (kF8 && kR >
   uint8_t* smem = align1024(smem_raw);
   uint8_t* sK = smem;                                   // stages of K tiles
   uint8_t* sV = sK + kStages * kTileB;                  // stages of V tiles
-  uint8_t* sVb = sV + kStages * kTileB;                 // e4m3 cache: the widened V tile (bf16)
-  uint8_t* sOnes = sVb + (kF8 ? kDecKvBytes : 0);       // [128][64] bf16 ones
+  uint8_t* sVb = sV + kStages * kTileB;                 // e4m3 cache: two widened V tiles (fp16)
+  uint8_t* sOnes = sVb + (kF8 ? 2 * kDecKvBytes : 0);   // [128][64] ones
   uint8_t* sP = sOnes + kDecKvBytes;                    // P^T
   uint8_t* sQ = sP + kDecPBytes;                        // Q rows (8 KB, 1024-aligned)
   DecCtl* ctl = reinterpret_cast<DecCtl*>(sQ + kDecQBytes);
@@ -278,7 +280,8 @@ __global__ void __launch_bounds__(kF8 ? kDecThreads8 : kDecThreads, (kF8 && kR >
   if (threadIdx.x == 0) {
     mbar_init(&ctl->q_full, 1);
     mbar_init(&ctl->q_conv, kDecTile);
-    mbar_init(&ctl->v_ready, kDecTile);
+    mbar_init(&ctl->v_ready[0], kDecTile);
+    mbar_init(&ctl->v_ready[1], kDecTile);
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&ctl->k_full[s], 1);
       mbar_init(&ctl->k_empty[s], kF8 ? kDecTile : 1);  // e4m3: freed by the 128 widening threads
@@ -291,7 +294,8 @@ __global__ void __launch_bounds__(kF8 ? kDecThreads8 : kDecThreads, (kF8 && kR >
       mbar_init(&ctl->kt_full[b], kDecTile);
     }
     mbar_init(&ctl->p_full, kDecTile);
-    mbar_init(&ctl->pv_done, 1);
+    mbar_init(&ctl->pv_done[0], 1);
+    mbar_init(&ctl->pv_done[1], 1);
     mbar_init(&ctl->o_full, 1);
     mbar_init(&ctl->sync, kDecTile);
     ctl->abort = 0;
@@ -382,14 +386,15 @@ __global__ void __launch_bounds__(kF8 ? kDecThreads8 : kDecThreads, (kF8 && kR >
         if (i >= 1) {
           const int j = i - 1;
           const int s = j % kStages;
-          // e4m3: V_j widened into the fp16 tile (v_ready).
+          // e4m3: V_j widened into fp16 tile j % 2 (v_ready).
           ok = mbar_wait(&ctl->p_full, j & 1, abort, &g_device_error, kDevErrTimeoutMma) &&
-               (kF8 ? mbar_wait(&ctl->v_ready, j & 1, abort, &g_device_error, kDevErrTimeoutMma)
+               (kF8 ? mbar_wait(&ctl->v_ready[j & 1], (j >> 1) & 1, abort, &g_device_error, kDevErrTimeoutMma)
                     : mbar_wait(&ctl->v_full[s], (j / kStages) & 1, abort, &g_device_error, kDevErrTimeoutMma));
           if (!ok) break;
           tc_fence_after();
-          dec_issue_pv<kF8>(tO, kF8 ? smem_u32(sVb) : smem_u32(sV + s * kDecKvBytes), ones_addr, p_addr, j > 0);
-          tc_commit(&ctl->pv_done);
+          dec_issue_pv<kF8>(tO, kF8 ? smem_u32(sVb + (j & 1) * kDecKvBytes) : smem_u32(sV + s * kDecKvBytes),
+                            ones_addr, p_addr, j > 0);
+          tc_commit(&ctl->pv_done[j & 1]);
           if constexpr (!kF8) tc_commit(&ctl->v_empty[s]);
         }
       }
@@ -433,11 +438,11 @@ __global__ void __launch_bounds__(kF8 ? kDecThreads8 : kDecThreads, (kF8 && kR >
         mbar_arrive(&ctl->k_empty[s]);
         tc_fence_before();
         mbar_arrive(&ctl->kt_full[b]);
-        // V_i -> the fp16 tile, whose last reader was the PV MMA of tile i-1.
-        // A slot that holds no token may hold any bits (NaN included) and
-        // its V row is still multiplied by P = 0: it becomes zeros.
-        if (i >= 1) {
-          ok = mbar_wait(&ctl->pv_done, (i - 1) & 1, abort, &g_device_error, kDevErrTimeoutDecode);
+        // V_i -> fp16 tile i % 2, whose last reader was the PV MMA of tile
+        // i-2.  A slot that holds no token may hold any bits (NaN included)
+        // and its V row is still multiplied by P = 0: it becomes zeros.
+        if (i >= 2) {
+          ok = mbar_wait(&ctl->pv_done[i & 1], ((i - 2) >> 1) & 1, abort, &g_device_error, kDevErrTimeoutDecode);
           if (!ok) break;
         }
         ok = mbar_wait(&ctl->v_full[s], (i / kStages) & 1, abort, &g_device_error, kDevErrTimeoutDecode);
@@ -450,14 +455,14 @@ __global__ void __launch_bounds__(kF8 ? kDecThreads8 : kDecThreads, (kF8 && kR >
 #pragma unroll
           for (int c = 0; c < 32; ++c) buf[c] = 0u;
         }
-        uint8_t* vline = sVb + (kl >> 3) * 1024 + (kl & 7) * 128;
+        uint8_t* vline = sVb + (i & 1) * kDecKvBytes + (kl >> 3) * 1024 + (kl & 7) * 128;
 #pragma unroll
         for (int c = 0; c < 8; ++c)
           *reinterpret_cast<uint4*>(vline + ((c ^ (kl & 7)) << 4)) =
               make_uint4(buf[4 * c], buf[4 * c + 1], buf[4 * c + 2], buf[4 * c + 3]);
         fence_proxy_async_smem();  // the fp16 tile for the MMA; the byte reads before the next TMA
         mbar_arrive(&ctl->v_empty[s]);
-        mbar_arrive(&ctl->v_ready);
+        mbar_arrive(&ctl->v_ready[i & 1]);
       }
     }
   } else {
@@ -533,7 +538,8 @@ __global__ void __launch_bounds__(kF8 ? kDecThreads8 : kDecThreads, (kF8 && kR >
       }
       // The previous PV read P^T and wrote O^T: wait for it before both.
       if (i > 0) {
-        ok = mbar_wait(&ctl->pv_done, (i - 1) & 1, abort, &g_device_error, kDevErrTimeoutDecode);
+        ok = mbar_wait(&ctl->pv_done[(i - 1) & 1], ((i - 1) >> 1) & 1, abort, &g_device_error,
+                       kDevErrTimeoutDecode);
         if (!ok) break;
         if (raise) {
           // O^T[lane][n] *= alpha[n]: head dims in lanes 0..63, row sums in
