@@ -20,7 +20,8 @@
 //   softmax over keys     one thread per key (its TMEM lane); the per-row
 //                         reference max is shared by all threads (seeded
 //                         with the sink logit, raised lazily: only when some
-//                         key exceeds it by more than 2^8, found by a vote)
+//                         key exceeds it by more than 2^8, found by an OR
+//                         over the keys in the barrier hardware)
 //   O^T += [V | 1]^T P^T  M = 128: rows 0..63 are the head dims (A = V read
 //                         MN-major), rows 64..127 multiply P^T by a tile of
 //                         ones and so accumulate the row sums l for free;
@@ -97,11 +98,9 @@ struct DecCtl {
   uint64_t pv_done[2];  // O^T += ... of tile i complete, barrier i % 2 (the softmax and the e4m3
                         // widening threads wait on different tiles' completions)
   uint64_t o_full;      // every MMA done
-  uint64_t sync;        // the 128 softmax threads
   float m_ref[kDecRows];    // reference max per query row (log2 units)
   float alpha[kDecRows];    // rescale factor of the current tile per row
   float wmax[4][kDecRows];  // per-warp tile maxima (rare path)
-  int vote[2][4];           // per-warp "a key exceeds the reference" flags, by tile parity
   uint32_t tmem_base;
   int abort;
 };
@@ -155,9 +154,16 @@ __device__ __forceinline__ DecWork dec_work(const DecParams& p) {
   return w;
 }
 
-// Position of the token in slot z (negative: the slot holds no token yet).
-__device__ __forceinline__ int dec_slot_pos(int z, int L, int C) {
-  int d = (L - 1 - z) % C;
+// Slot of the newest token, (L - 1) mod C (one division per CTA).
+__device__ __forceinline__ int dec_last_slot(int L, int C) {
+  int r = (L - 1) % C;
+  return r < 0 ? r + C : r;
+}
+
+// Position of the token in slot z, 0 <= z < C (negative: the slot holds no
+// token yet): the largest position <= L - 1 that is congruent to z mod C.
+__device__ __forceinline__ int dec_slot_pos(int z, int L, int last_slot, int C) {
+  int d = last_slot - z;
   if (d < 0) d += C;
   return L - 1 - d;
 }
@@ -191,11 +197,16 @@ __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t codes) {
   return h2;
 }
 
-// One cache row of 64 e4m3 codes -> 32 packed fp16 pairs (element order kept).
-__device__ __forceinline__ void dec_row_e4m3_to_f16(const uint8_t* src, uint32_t* out) {
+// Row r of a byte tile (64 e4m3 codes) -> 32 packed fp16 pairs (element order
+// kept).  The tile was written by TMA with the 64-byte swizzle: 16-byte chunk
+// c of row r sits at chunk c ^ ((r >> 1) & 3), so the eight rows that one
+// quarter-warp reads fall in eight different bank groups.
+__device__ __forceinline__ void dec_row_e4m3_to_f16(const uint8_t* tile, int r, uint32_t* out) {
+  const uint4* row = reinterpret_cast<const uint4*>(tile + r * kHeadDim);
+  const int swz = (r >> 1) & 3;
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
-    const uint4 v = reinterpret_cast<const uint4*>(src)[q];
+    const uint4 v = row[q ^ swz];
     const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
@@ -231,12 +242,22 @@ __device__ __forceinline__ void dec_issue_pv(uint32_t tmem_o, uint32_t v_addr, u
   }
 }
 
-__device__ __forceinline__ bool dec_group_sync(DecCtl* ctl, uint32_t& phase, volatile int* abort) {
-  mbar_arrive(&ctl->sync);
-  const bool ok = mbar_wait(&ctl->sync, phase, abort, &g_device_error, kDevErrTimeoutDecode);
-  phase ^= 1u;
-  return ok;
+// The 128 softmax threads (warps 0-3) on hardware barrier 1: an OR of one
+// predicate over them, and a plain barrier.  Every softmax thread executes the
+// same sequence of these (see the softmax loop), so none is left waiting.
+__device__ __forceinline__ bool dec_group_any(bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred pi, po;\n\t"
+      "setp.ne.u32 pi, %1, 0;\n\t"
+      "bar.red.or.pred po, 1, %2, pi;\n\t"
+      "selp.u32 %0, 1, 0, po;\n\t}"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(pred)), "n"(kDecTile)
+      : "memory");
+  return r != 0;
 }
+__device__ __forceinline__ void dec_group_sync() { named_barrier(1, kDecTile); }
 
 // Loads / stores kN (16, 32 or 64) consecutive TMEM columns of this warp's lanes.
 template <int kN>
@@ -297,7 +318,6 @@ __global__ void __launch_bounds__(kF8 ? kDecThreads8 : kDecThreads, (kF8 && kR >
     mbar_init(&ctl->pv_done[0], 1);
     mbar_init(&ctl->pv_done[1], 1);
     mbar_init(&ctl->o_full, 1);
-    mbar_init(&ctl->sync, kDecTile);
     ctl->abort = 0;
     if (w.bad) atomicCAS(&g_device_error, 0, static_cast<int>(kDevErrDecodeCacheTooSmall));
     fence_mbar_init();
@@ -405,6 +425,7 @@ __global__ void __launch_bounds__(kF8 ? kDecThreads8 : kDecThreads, (kF8 && kR >
     if constexpr (kF8) {
       const int kl = 32 * (warp & 3) + (threadIdx.x & 31);  // slot == the TMEM lane this warp may access
       const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+      const int last_slot = dec_last_slot(w.L, p.C);
       bool ok = true;
       if (w.n > 0) {
         // Q (bf16, as loaded) -> fp16 in place: elementwise, so the swizzle
@@ -429,7 +450,7 @@ __global__ void __launch_bounds__(kF8 ? kDecThreads8 : kDecThreads, (kF8 && kR >
         }
         ok = mbar_wait(&ctl->k_full[s], (i / kStages) & 1, abort, &g_device_error, kDevErrTimeoutDecode);
         if (!ok) break;
-        dec_row_e4m3_to_f16(sK + s * kTileB + kl * kHeadDim, buf);
+        dec_row_e4m3_to_f16(sK + s * kTileB, kl, buf);
         tmem_st32(tmem + lane_base + kDecTmemK + 32 * b, buf);
         // Release the byte stage only after its values have been consumed
         // (a shared load may still be in flight until its result is used),
@@ -448,9 +469,9 @@ __global__ void __launch_bounds__(kF8 ? kDecThreads8 : kDecThreads, (kF8 && kR >
         ok = mbar_wait(&ctl->v_full[s], (i / kStages) & 1, abort, &g_device_error, kDevErrTimeoutDecode);
         if (!ok) break;
         const int z = w.z0 + i * kDecTile + kl;
-        const int pos = z < p.C ? dec_slot_pos(z, w.L, p.C) : -1;
+        const int pos = z < p.C ? dec_slot_pos(z, w.L, last_slot, p.C) : -1;
         if (pos >= 0) {
-          dec_row_e4m3_to_f16(sV + s * kTileB + kl * kHeadDim, buf);
+          dec_row_e4m3_to_f16(sV + s * kTileB, kl, buf);
         } else {
 #pragma unroll
           for (int c = 0; c < 32; ++c) buf[c] = 0u;
@@ -471,40 +492,63 @@ __global__ void __launch_bounds__(kF8 ? kDecThreads8 : kDecThreads, (kF8 && kR >
     const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
     // e4m3: logits carry k_scale, O carries v_scale.
     const float sl2 = kF8 ? p.scale_log2 * __ldg(p.k_scale + w.g) : p.scale_log2;
-    uint32_t sync_phase = 0;
+    const int last_slot = dec_last_slot(w.L, p.C);
+    // The reference max of each row, also kept in registers (it changes only
+    // when raised, below); kR = 64 reads it from shared memory instead.
+    float mreg[kR <= 32 ? kR : 1];
+    if constexpr (kR <= 32) {
+#pragma unroll
+      for (int n = 0; n < kR; ++n) mreg[n] = ctl->m_ref[n];
+    }
+    auto mref = [&](int n) -> float {
+      if constexpr (kR <= 32) return mreg[n];
+      else return ctl->m_ref[n];
+    };
+    // Every softmax thread runs all w.n iterations and meets the other 127 at
+    // the group barrier once per tile (three times on a raise), also after an
+    // abort: then it only skips the work, so no barrier is left waiting.
+    // Wait outcomes are made warp-uniform for the .sync.aligned TMEM ops.
     bool ok = true;
-    for (int i = 0; ok && i < w.n; ++i) {
+    for (int i = 0; i < w.n; ++i) {
       const int b = i & 1;
-      ok = mbar_wait(&ctl->s_full[b], (i >> 1) & 1, abort, &g_device_error, kDevErrTimeoutDecode);
-      if (!ok) break;
-      tc_fence_after();
+      if (ok) ok = mbar_wait(&ctl->s_full[b], (i >> 1) & 1, abort, &g_device_error, kDevErrTimeoutDecode);
+      ok = __all_sync(0xffffffffu, ok);
       float x[kR];
-      {
+      if (ok) {
+        tc_fence_after();
         uint32_t raw[kR];
         dec_tmem_ld<kR>(tmem + lane_base + kDecTmemS + b * kDecRows, raw);
 #pragma unroll
         for (int n = 0; n < kR; ++n) x[n] = __uint_as_float(raw[n]);
+        tc_fence_before();
+        mbar_arrive(&ctl->s_free[b]);
+      } else {
+#pragma unroll
+        for (int n = 0; n < kR; ++n) x[n] = -INFINITY;
       }
-      tc_fence_before();
-      mbar_arrive(&ctl->s_free[b]);
-      // Mask: slot -> position -> allowed for each query row.
+      // Mask: slot -> position -> the query rows that see it.  New token t
+      // (position L0 + t, rows t*G .. t*G + G - 1) sees position pos iff
+      // pos <= L0 + t and, with a window, L0 + t - pos < window: one range of
+      // tokens, hence one range [n_lo, n_lo + n_span) of rows.
       const int z = w.z0 + i * kDecTile + kl;
-      const int pos = z < p.C ? dec_slot_pos(z, w.L, p.C) : -1;
+      const int pos = z < p.C ? dec_slot_pos(z, w.L, last_slot, p.C) : -1;
+      int n_lo = 0, n_span = 0;
+      if (pos >= 0) {
+        const int t_lo = max(0, pos - w.L0);
+        const int t_hi = p.window > 0 ? min(p.Lq, pos - w.L0 + p.window) : p.Lq;
+        n_lo = t_lo * p.G;
+        n_span = max(0, t_hi * p.G - n_lo);
+      }
       bool viol = false;
 #pragma unroll
       for (int n = 0; n < kR; ++n) {
-        const int qi = w.L0 + (n >> p.G_log2);  // query position of row n
-        const bool allowed = n < p.R && pos >= 0 && pos <= qi && (p.window <= 0 || qi - pos < p.window);
+        const bool allowed = static_cast<unsigned>(n - n_lo) < static_cast<unsigned>(n_span);
         x[n] = allowed ? x[n] * sl2 : -INFINITY;
-        viol |= x[n] > ctl->m_ref[n] + kDecRescaleLog2;
+        viol |= x[n] > mref(n) + kDecRescaleLog2;
       }
-      // Raise the shared reference max only when some key exceeds it by
-      // more than 2^8 (decided by a vote of all 128 keys).
-      const unsigned any_w = __ballot_sync(0xffffffffu, viol);
-      if ((kl & 31) == 0) ctl->vote[b][warp] = any_w != 0u;
-      ok = dec_group_sync(ctl, sync_phase, abort);
-      if (!ok) break;
-      const bool raise = ctl->vote[b][0] | ctl->vote[b][1] | ctl->vote[b][2] | ctl->vote[b][3];
+      // Raise the reference max only when some key exceeds it by more than
+      // 2^8: an OR over the 128 keys, taken in the barrier hardware.
+      const bool raise = dec_group_any(viol);
       if (raise) {
 #pragma unroll
         for (int n = 0; n < kR; ++n) {
@@ -515,8 +559,7 @@ __global__ void __launch_bounds__(kF8 ? kDecThreads8 : kDecThreads, (kF8 && kR >
             if ((kl & 31) == 0) ctl->wmax[warp][n] = v;
           }
         }
-        ok = dec_group_sync(ctl, sync_phase, abort);
-        if (!ok) break;
+        dec_group_sync();
         if (kl < p.R) {
           const float tmax = fmaxf(fmaxf(ctl->wmax[0][kl], ctl->wmax[1][kl]), fmaxf(ctl->wmax[2][kl], ctl->wmax[3][kl]));
           const float mr = ctl->m_ref[kl];
@@ -524,23 +567,27 @@ __global__ void __launch_bounds__(kF8 ? kDecThreads8 : kDecThreads, (kF8 && kR >
           ctl->alpha[kl] = up ? ex2_approx(mr - tmax) : 1.f;
           if (up) ctl->m_ref[kl] = tmax;
         }
-        ok = dec_group_sync(ctl, sync_phase, abort);
-        if (!ok) break;
+        dec_group_sync();
+        if constexpr (kR <= 32) {
+#pragma unroll
+          for (int n = 0; n < kR; ++n) mreg[n] = ctl->m_ref[n];
+        }
       }
+      if (!ok) continue;
       // P^T row of this key, packed to bf16 pairs (rows 2c, 2c+1).
       uint32_t pk[kR / 2];
 #pragma unroll
       for (int c = 0; c < kR / 2; ++c) {
-        const float m0 = ctl->m_ref[2 * c], m1 = ctl->m_ref[2 * c + 1];
+        const float m0 = mref(2 * c), m1 = mref(2 * c + 1);
         const float e0 = ex2_approx(x[2 * c] - (m0 == -INFINITY ? 0.f : m0));
         const float e1 = ex2_approx(x[2 * c + 1] - (m1 == -INFINITY ? 0.f : m1));
         pk[c] = kF8 ? pack_f16x2(e0, e1) : pack_bf16x2(e0, e1);
       }
       // The previous PV read P^T and wrote O^T: wait for it before both.
       if (i > 0) {
-        ok = mbar_wait(&ctl->pv_done[(i - 1) & 1], ((i - 1) >> 1) & 1, abort, &g_device_error,
-                       kDevErrTimeoutDecode);
-        if (!ok) break;
+        ok = __all_sync(0xffffffffu, mbar_wait(&ctl->pv_done[(i - 1) & 1], ((i - 1) >> 1) & 1, abort,
+                                               &g_device_error, kDevErrTimeoutDecode));
+        if (!ok) continue;
         if (raise) {
           // O^T[lane][n] *= alpha[n]: head dims in lanes 0..63, row sums in
           // lanes 64..127, query rows in columns.
@@ -555,13 +602,16 @@ __global__ void __launch_bounds__(kF8 ? kDecThreads8 : kDecThreads, (kF8 && kR >
       // A slot that holds no token (never written, or past this sequence's
       // C slots) may hold any bits, NaN included, and its V row is still
       // multiplied by P = 0: its row of the V operand is zeroed.
-      if (!kF8 && pos < 0) {
+      if (!kF8 && __any_sync(0xffffffffu, pos < 0)) {
         const int sv = i % kStages;
-        ok = mbar_wait(&ctl->v_full[sv], (i / kStages) & 1, abort, &g_device_error, kDevErrTimeoutDecode);
-        if (!ok) break;
-        uint4* vrow = reinterpret_cast<uint4*>(sV + sv * kDecKvBytes + (kl >> 3) * 1024 + (kl & 7) * 128);
+        ok = __all_sync(0xffffffffu, mbar_wait(&ctl->v_full[sv], (i / kStages) & 1, abort, &g_device_error,
+                                               kDevErrTimeoutDecode));
+        if (!ok) continue;
+        if (pos < 0) {
+          uint4* vrow = reinterpret_cast<uint4*>(sV + sv * kDecKvBytes + (kl >> 3) * 1024 + (kl & 7) * 128);
 #pragma unroll
-        for (int c = 0; c < 8; ++c) vrow[c] = make_uint4(0u, 0u, 0u, 0u);
+          for (int c = 0; c < 8; ++c) vrow[c] = make_uint4(0u, 0u, 0u, 0u);
+        }
       }
       // P^T [slot kl][rows]: 128 B per slot, 16-byte chunk c (rows 8c..8c+7)
       // at chunk position c ^ (kl % 8).
@@ -581,6 +631,7 @@ __global__ void __launch_bounds__(kF8 ? kDecThreads8 : kDecThreads, (kF8 && kR >
     const size_t cta = static_cast<size_t>(blockIdx.x);
     bool have = ok && w.n > 0;
     if (have) have = mbar_wait(&ctl->o_full, 0, abort, &g_device_error, kDevErrTimeoutEpilogue);
+    have = __all_sync(0xffffffffu, have);
     if (have) tc_fence_after();
     if (warp < 3) {
       uint32_t o[kR];

@@ -60,8 +60,10 @@ inline bool make_map_3d_f32(CUtensorMap* map, const void* base, int inner, int m
   return r == CUDA_SUCCESS;
 }
 
-// 3-D byte view [outer][mid][inner] (e.g. an e4m3 cache), no swizzle: a box
-// lands in shared memory as plain rows of `inner` bytes.
+// 3-D byte view [outer][mid][inner] (e.g. an e4m3 cache) with inner = 64: a
+// box lands in shared memory as rows of 64 bytes under the 64-byte swizzle
+// (16-byte chunk c of row r at chunk c ^ ((r >> 1) & 3); the destination must
+// be 512-byte aligned).
 inline bool make_map_3d_u8(CUtensorMap* map, const void* base, int inner, int mid, int outer, int box_mid,
                            int box_outer) {
   EncodeTiledFn enc = get_encode_tiled();
@@ -73,7 +75,7 @@ inline bool make_map_3d_u8(CUtensorMap* map, const void* base, int inner, int mi
                        static_cast<cuuint32_t>(box_outer)};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
