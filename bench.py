@@ -198,9 +198,11 @@ def measured_traffic():
 
 # --------------------------------------------------------------- decode
 DECODE_CASES = (
-    # (name, sequences, cached tokens, new tokens, cache slots, window)
-    ("decode 64 seqs x 8191 cached + 1 new, full-causal layer, linear 8192-slot cache", 64, 8191, 1, 8192, 0),
-    ("decode 64 seqs x 8191 cached + 1 new, window-128 layer, 128-slot ring", 64, 8191, 1, 128, 128),
+    # (name, sequences, cached tokens, new tokens, cache slots, window, e4m3 cache)
+    ("decode 64 seqs x 8191 cached + 1 new, full-causal layer, linear 8192-slot cache", 64, 8191, 1, 8192, 0, False),
+    ("decode 64 seqs x 8191 cached + 1 new, window-128 layer, 128-slot ring", 64, 8191, 1, 128, 128, False),
+    ("decode 64 seqs x 8191 cached + 1 new, full-causal layer, linear 8192-slot e4m3 cache", 64, 8191, 1, 8192, 0,
+     True),
 )
 
 
@@ -212,12 +214,20 @@ def measure_decode(torch, ops, stream, iters=20):
     _, hbm, kind = read_peaks()
     res = []
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
-    for name, Bd, L0, Lq, C, W in DECODE_CASES:
+    for name, Bd, L0, Lq, C, W, f8 in DECODE_CASES:
         a = synth.decode_inputs(7, [0], Lq, HQ, HKV)  # sinks and new-token rows
         g = torch.Generator(device="cuda").manual_seed(7)
         mk = lambda *shape: torch.randn(*shape, device="cuda", generator=g).to(torch.bfloat16)  # noqa: E731
         q, kn, vn = mk(Bd, Lq, HQ, D), mk(Bd, Lq, HKV, D), mk(Bd, Lq, HKV, D)
-        kc, vc = mk(Bd, C, HKV, D), mk(Bd, C, HKV, D)
+        if f8:
+            # e4m3 codes of both signs, NaN codes (0x7F, 0xFF) excluded; one scale per KV head
+            codes = lambda: (torch.randint(0, 0x7F, (Bd, C, HKV, D), dtype=torch.uint8, device="cuda", generator=g)  # noqa: E731
+                             | (torch.randint(0, 2, (Bd, C, HKV, D), dtype=torch.uint8, device="cuda", generator=g) << 7))
+            kc, vc = codes(), codes()
+            k_scale = torch.full((HKV,), 1.0 / 64, dtype=torch.float32, device="cuda")
+            v_scale = torch.full((HKV,), 1.0 / 64, dtype=torch.float32, device="cuda")
+        else:
+            kc, vc = mk(Bd, C, HKV, D), mk(Bd, C, HKV, D)
         sl = torch.full((Bd,), L0, dtype=torch.int32, device="cuda")
         sinks = torch.from_numpy(a["sinks"]).cuda()
         ws = torch.empty((ops.decode_workspace_size(Bd, Lq, C, L0 + Lq, HQ, HKV, W),), dtype=torch.uint8,
@@ -226,8 +236,12 @@ def measure_decode(torch, ops, stream, iters=20):
         lse = torch.empty((HQ, Bd * Lq), dtype=torch.float32, device="cuda")
 
         def call():
-            ops.decode(q, kn, vn, kc, vc, sl, sinks, W, 0.125, max_seqlen=L0 + Lq, out=out, lse=lse, workspace=ws,
-                       stream=stream)
+            if f8:
+                ops.decode_e4m3(q, kn, vn, kc, vc, sl, k_scale, v_scale, sinks, W, 0.125, max_seqlen=L0 + Lq, out=out,
+                                lse=lse, workspace=ws, stream=stream)
+            else:
+                ops.decode(q, kn, vn, kc, vc, sl, sinks, W, 0.125, max_seqlen=L0 + Lq, out=out, lse=lse,
+                           workspace=ws, stream=stream)
         for _ in range(3):
             call()
         torch.cuda.synchronize()
@@ -244,7 +258,7 @@ def measure_decode(torch, ops, stream, iters=20):
             raise RuntimeError("a decode kernel reported an error")
         ms = tot / iters
         keys = min(L0 + Lq, C) if W <= 0 else min(L0 + Lq, W + Lq - 1, C)
-        kv = Bd * keys * HKV * D * 2 * 2
+        kv = Bd * keys * HKV * D * 2 * (1 if f8 else 2)  # K and V bytes as stored
         res.append({"workload": name, "us": ms * 1e3, "kv_bytes": kv, "achieved_GBps": kv / ms / 1e6,
                     "peak_GBps": hbm, "frac": kv / ms / 1e6 / hbm, "peak_source": f"{kind} hbm_gbs",
                     "launches": ops.decode_launches(Bd, Lq, C, L0 + Lq, HQ, HKV)})

@@ -197,17 +197,22 @@ __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t codes) {
   return h2;
 }
 
-// Row r of a byte tile (64 e4m3 codes) -> 32 packed fp16 pairs (element order
-// kept).  The tile was written by TMA with the 64-byte swizzle: 16-byte chunk
-// c of row r sits at chunk c ^ ((r >> 1) & 3), so the eight rows that one
-// quarter-warp reads fall in eight different bank groups.
-__device__ __forceinline__ void dec_row_e4m3_to_f16(const uint8_t* tile, int r, uint32_t* out) {
+// Row r of a byte tile (64 e4m3 codes) into registers, in element order.  The
+// tile was written by TMA with the 64-byte swizzle: 16-byte chunk c of row r
+// sits at chunk c ^ ((r >> 1) & 3), so the eight rows that one quarter-warp
+// reads fall in eight different bank groups.
+__device__ __forceinline__ void dec_row_load(const uint8_t* tile, int r, uint4* raw) {
   const uint4* row = reinterpret_cast<const uint4*>(tile + r * kHeadDim);
   const int swz = (r >> 1) & 3;
 #pragma unroll
+  for (int q = 0; q < 4; ++q) raw[q] = row[q ^ swz];
+}
+
+// 64 e4m3 codes -> 32 packed fp16 pairs (element order kept).
+__device__ __forceinline__ void dec_row_widen(const uint4* raw, uint32_t* out) {
+#pragma unroll
   for (int q = 0; q < 4; ++q) {
-    const uint4 v = row[q ^ swz];
-    const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+    const uint32_t w4[4] = {raw[q].x, raw[q].y, raw[q].z, raw[q].w};
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       out[8 * q + 2 * u] = e4m3x2_to_f16x2(w4[u]);
@@ -259,16 +264,19 @@ __device__ __forceinline__ bool dec_group_any(bool pred) {
 }
 __device__ __forceinline__ void dec_group_sync() { named_barrier(1, kDecTile); }
 
-// Loads / stores kN (16, 32 or 64) consecutive TMEM columns of this warp's lanes.
+// Loads / stores kN (8, 16, 32 or 64) consecutive TMEM columns of this warp's lanes.
 template <int kN>
 __device__ __forceinline__ void dec_tmem_ld(uint32_t taddr, uint32_t* r) {
-  if constexpr (kN == 16) tmem_ld16(taddr, r);
+  if constexpr (kN == 8) tmem_ld8(taddr, r);
+  else if constexpr (kN == 16) tmem_ld16(taddr, r);
   else if constexpr (kN == 32) tmem_ld32(taddr, r);
   else tmem_ld64(taddr, r);
 }
 template <int kN>
 __device__ __forceinline__ void dec_tmem_st(uint32_t taddr, const uint32_t* r) {
-  if constexpr (kN == 16) {
+  if constexpr (kN == 8) {
+    tmem_st8(taddr, r);
+  } else if constexpr (kN == 16) {
     tmem_st16(taddr, r);
   } else {
 #pragma unroll
@@ -276,7 +284,7 @@ __device__ __forceinline__ void dec_tmem_st(uint32_t taddr, const uint32_t* r) {
   }
 }
 
-// kR: query rows handled in registers (16, 32 or 64; >= G * Lq).
+// kR: query rows handled in registers (8, 16, 32 or 64; >= G * Lq).
 // kF8: the cache holds e4m3 codes (see the file comment).
 template <int kR, bool kF8>
 __global__ void __launch_bounds__(kF8 ? kDecThreads8 : kDecThreads, (kF8 && kR > 16) ? 1 : 2)
@@ -450,7 +458,9 @@ __global__ void __launch_bounds__(kF8 ? kDecThreads8 : kDecThreads, (kF8 && kR >
         }
         ok = mbar_wait(&ctl->k_full[s], (i / kStages) & 1, abort, &g_device_error, kDevErrTimeoutDecode);
         if (!ok) break;
-        dec_row_e4m3_to_f16(sK + s * kTileB, kl, buf);
+        uint4 raw[4];
+        dec_row_load(sK + s * kTileB, kl, raw);
+        dec_row_widen(raw, buf);
         tmem_st32(tmem + lane_base + kDecTmemK + 32 * b, buf);
         // Release the byte stage only after its values have been consumed
         // (a shared load may still be in flight until its result is used),
@@ -471,7 +481,8 @@ __global__ void __launch_bounds__(kF8 ? kDecThreads8 : kDecThreads, (kF8 && kR >
         const int z = w.z0 + i * kDecTile + kl;
         const int pos = z < p.C ? dec_slot_pos(z, w.L, last_slot, p.C) : -1;
         if (pos >= 0) {
-          dec_row_e4m3_to_f16(sV + s * kTileB, kl, buf);
+          dec_row_load(sV + s * kTileB, kl, raw);
+          dec_row_widen(raw, buf);
         } else {
 #pragma unroll
           for (int c = 0; c < 32; ++c) buf[c] = 0u;
@@ -511,6 +522,20 @@ __global__ void __launch_bounds__(kF8 ? kDecThreads8 : kDecThreads, (kF8 && kR >
     bool ok = true;
     for (int i = 0; i < w.n; ++i) {
       const int b = i & 1;
+      // Mask: slot -> position -> the query rows that see it.  New token t
+      // (position L0 + t, rows t*G .. t*G + G - 1) sees position pos iff
+      // pos <= L0 + t and, with a window, L0 + t - pos < window: one range of
+      // tokens, hence one range [n_lo, n_lo + n_span) of rows.
+      const int z = w.z0 + i * kDecTile + kl;
+      const int pos = z < p.C ? dec_slot_pos(z, w.L, last_slot, p.C) : -1;
+      int n_lo = 0, n_span = 0;  // (computed before the wait for S, which it overlaps)
+      if (pos >= 0) {
+        const int t_lo = max(0, pos - w.L0);
+        const int t_hi = p.window > 0 ? min(p.Lq, pos - w.L0 + p.window) : p.Lq;
+        n_lo = t_lo * p.G;
+        n_span = max(0, t_hi * p.G - n_lo);
+      }
+      asm volatile("" ::"r"(n_lo), "r"(n_span));
       if (ok) ok = mbar_wait(&ctl->s_full[b], (i >> 1) & 1, abort, &g_device_error, kDevErrTimeoutDecode);
       ok = __all_sync(0xffffffffu, ok);
       float x[kR];
@@ -525,19 +550,6 @@ __global__ void __launch_bounds__(kF8 ? kDecThreads8 : kDecThreads, (kF8 && kR >
       } else {
 #pragma unroll
         for (int n = 0; n < kR; ++n) x[n] = -INFINITY;
-      }
-      // Mask: slot -> position -> the query rows that see it.  New token t
-      // (position L0 + t, rows t*G .. t*G + G - 1) sees position pos iff
-      // pos <= L0 + t and, with a window, L0 + t - pos < window: one range of
-      // tokens, hence one range [n_lo, n_lo + n_span) of rows.
-      const int z = w.z0 + i * kDecTile + kl;
-      const int pos = z < p.C ? dec_slot_pos(z, w.L, last_slot, p.C) : -1;
-      int n_lo = 0, n_span = 0;
-      if (pos >= 0) {
-        const int t_lo = max(0, pos - w.L0);
-        const int t_hi = p.window > 0 ? min(p.Lq, pos - w.L0 + p.window) : p.Lq;
-        n_lo = t_lo * p.G;
-        n_span = max(0, t_hi * p.G - n_lo);
       }
       bool viol = false;
 #pragma unroll

@@ -378,11 +378,13 @@ sink_attn_status decode_impl(const sink_attn_decode_dims* d, const void* q, cons
   }
   // Register arrays sized for the real query rows.
   using Kern = void (*)(CUtensorMap, CUtensorMap, CUtensorMap, DecParams);
-  static const Kern kerns[2][3] = {
-      {sink_attn_decode_kernel<16, false>, sink_attn_decode_kernel<32, false>, sink_attn_decode_kernel<64, false>},
-      {sink_attn_decode_kernel<16, true>, sink_attn_decode_kernel<32, true>, sink_attn_decode_kernel<64, true>}};
-  static int smem_set[2][3] = {{0, 0, 0}, {0, 0, 0}};
-  const int vi = p.R <= 16 ? 0 : (p.R <= 32 ? 1 : 2);
+  static const Kern kerns[2][4] = {
+      {sink_attn_decode_kernel<8, false>, sink_attn_decode_kernel<16, false>, sink_attn_decode_kernel<32, false>,
+       sink_attn_decode_kernel<64, false>},
+      {sink_attn_decode_kernel<8, true>, sink_attn_decode_kernel<16, true>, sink_attn_decode_kernel<32, true>,
+       sink_attn_decode_kernel<64, true>}};
+  static int smem_set[2][4] = {{0, 0, 0, 0}, {0, 0, 0, 0}};
+  const int vi = p.R <= 8 ? 0 : (p.R <= 16 ? 1 : (p.R <= 32 ? 2 : 3));
   const Kern kern = kerns[e4m3][vi];
   const size_t smem = e4m3 ? kDecSmemBytes8 : kDecSmemBytes;
   if (!set_smem_once(kern, smem, &smem_set[e4m3][vi])) return SINK_ATTN_ERR_CUDA;

@@ -35,6 +35,26 @@ __device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t* r) {
       : "r"(taddr)
       : "memory");
 }
+// Loads 8 consecutive 32-bit TMEM columns of this warp's 32 lanes (one lane
+// per thread) and waits for them, so the registers are valid on return.
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];\n\t"
+      "tcgen05.wait::ld.sync.aligned;\n"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+      : "r"(taddr)
+      : "memory");
+}
+// Stores 8 consecutive 32-bit TMEM columns of this warp's 32 lanes and waits
+// until the stores are done.
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};\n\t"
+      "tcgen05.wait::st.sync.aligned;\n"
+      :
+      : "r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+      : "memory");
+}
 // Stores 16 consecutive 32-bit TMEM columns of this warp's 32 lanes and
 // waits until the stores are done (the source registers are free again).
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
