@@ -316,11 +316,12 @@ __device__ __forceinline__ uint32_t ds_smem_offset(int key, int chunk16) {
 }
 
 // P^T for this thread's key over the 64 query rows [64*ch, 64*ch+64) of a
-// tile: P = 2^(S^T * scale*log2e - lse2), zero where the pair is masked,
-// rounded to bf16 and packed in row pairs (pk[r/2] holds rows r, r+1).  The
-// scaling runs two rows per instruction (a.lse2 holds -lse2).
+// tile: P = 2^(S^T * scale*log2e - lse2), zero outside the rows
+// [r_lo, r_lo + r_span) that see the key (kMask), rounded to bf16 and packed
+// in row pairs (pk[r/2] holds rows r, r+1).  The scaling runs two rows per
+// instruction (a.lse2 holds -lse2).
 template <bool kMask>
-__device__ __forceinline__ void bwd_p_rows(uint32_t tS, const BwdAux& a, int ch, float sl2, int j, int q0, int G_log2,
+__device__ __forceinline__ void bwd_p_rows(uint32_t tS, const BwdAux& a, int ch, float sl2, int r_lo, int r_span,
                                            uint32_t* pk) {
   const uint64_t sl2x2 = f32x2_pack(sl2, sl2);
 #pragma unroll
@@ -341,10 +342,7 @@ __device__ __forceinline__ void bwd_p_rows(uint32_t tS, const BwdAux& a, int ch,
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         pe[u] = ex2_approx(y[u]);
-        if (kMask) {
-          const int pos = (col + u) >> G_log2;
-          if (!(j >= a.lo[pos] && j <= q0 + pos)) pe[u] = 0.f;
-        }
+        if (kMask && static_cast<unsigned>(col + u - r_lo) >= static_cast<unsigned>(r_span)) pe[u] = 0.f;
       }
       pk[16 * half + c / 2] = pack_bf16x2(pe[0], pe[1]);
       pk[16 * half + c / 2 + 1] = pack_bf16x2(pe[2], pe[3]);
@@ -521,6 +519,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const int j = w.k0 + kl;                 // this thread's key
     const uint32_t lane_base = static_cast<uint32_t>(32 * lg) << 16;
     const float sl2 = p.scale_log2;
+    // The tokens that see key j are j <= t <= t_max (the end of j's document
+    // and, with a window, j + W - 1), so in every query tile the rows that
+    // see it form one range: the mask is one unsigned compare per element.
+    int t_max = -1;
+    if (j < geo.T) {
+      t_max = doc_end(geo, j) - 1;
+      if (geo.window > 0) t_max = min(t_max, j + geo.window - 1);
+    }
+    const int G = 1 << geo.G_log2;
     bool ok = true;
     for (int i = 0; i < w.nq; ++i) {
       const int st = i % kBwdStages;
@@ -539,10 +546,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const uint32_t tDP = tmem + lane_base + kBwdTmemDP + 64 * ch;
       uint32_t pk[32];
       // The mask test is resolved once per tile (CTA-uniform), not per element.
-      if (full)
-        bwd_p_rows<false>(tS, a, ch, sl2, j, q0, geo.G_log2, pk);
-      else
-        bwd_p_rows<true>(tS, a, ch, sl2, j, q0, geo.G_log2, pk);
+      if (full) {
+        bwd_p_rows<false>(tS, a, ch, sl2, 0, 0, pk);
+      } else {
+        const int r_lo = (max(j, q0) - q0) * G;
+        const int r_span = max(0, (min(t_max, q_last) - q0 + 1) * G - r_lo);
+        bwd_p_rows<true>(tS, a, ch, sl2, r_lo, r_span, pk);
+      }
       // P^T (bf16) of this warp's 64 rows over the first half of its own
       // S^T columns (rows 0-63 -> columns 0..31, rows 64-127 -> 64..95):
       // this warp has read them and no other warp reads them.
