@@ -168,10 +168,13 @@ __device__ __forceinline__ int dec_slot_pos(int z, int L, int last_slot, int C) 
   return L - 1 - d;
 }
 
-// S^T (64 columns) = K Q^T: A = the K tile (128 slots, K-major), B = Q
-// (64 rows, K-major).
+// S^T (kN columns) = K Q^T: A = the K tile (128 slots, K-major), B = the
+// first kN rows of Q (K-major).  kN = max(kR, 16), the smallest N an M = 128
+// MMA of this kind takes: the operand reads and the MMA time follow the real
+// query rows, not the 64 rows the tiles are laid out for.
+template <int kN>
 __device__ __forceinline__ void dec_issue_qk(uint32_t tmem_s, uint32_t k_addr, uint32_t q_addr) {
-  constexpr uint32_t idesc = make_idesc_bf16(kDecTile, kDecRows, 0, 0);
+  constexpr uint32_t idesc = make_idesc_bf16(kDecTile, kN, 0, 0);
 #pragma unroll
   for (int kk = 0; kk < kHeadDim / 16; ++kk) {
     const uint64_t a = make_sdesc_sw128(k_addr + kk * 32, 16, 1024);
@@ -181,8 +184,9 @@ __device__ __forceinline__ void dec_issue_qk(uint32_t tmem_s, uint32_t k_addr, u
 }
 
 // S^T = K Q^T in fp16 with K (32 packed columns) read from TMEM.
+template <int kN>
 __device__ __forceinline__ void dec_issue_qk_ts(uint32_t tmem_s, uint32_t tmem_k, uint32_t q_addr) {
-  constexpr uint32_t idesc = make_idesc_f16(kDecTile, kDecRows, 0, 0);
+  constexpr uint32_t idesc = make_idesc_f16(kDecTile, kN, 0, 0);
 #pragma unroll
   for (int kk = 0; kk < kHeadDim / 16; ++kk) {
     const uint64_t b = make_sdesc_sw128(q_addr + kk * 32, 16, 1024);
@@ -231,13 +235,13 @@ __device__ __forceinline__ uint32_t bf16x2_to_f16x2_sat(uint32_t v) {
 
 // O^T (+)= [V | 1]^T P^T over the 128 slots of a tile: A (M = 128) is read
 // MN-major from the V tile (M rows 0..63) and the ones tile (M rows 64..127,
-// reached through the descriptor's leading-byte offset); B = P^T [slots][64
-// rows], MN-major.
-template <bool kF16>
+// reached through the descriptor's leading-byte offset); B = the first kN
+// query rows of P^T [slots][64 rows], MN-major.
+template <bool kF16, int kN>
 __device__ __forceinline__ void dec_issue_pv(uint32_t tmem_o, uint32_t v_addr, uint32_t ones_addr, uint32_t p_addr,
                                              bool accumulate) {
   constexpr uint32_t idesc =
-      kF16 ? make_idesc_f16(kDecTile, kDecRows, 1, 1) : make_idesc_bf16(kDecTile, kDecRows, 1, 1);
+      kF16 ? make_idesc_f16(kDecTile, kN, 1, 1) : make_idesc_bf16(kDecTile, kN, 1, 1);
   const uint32_t lbo = ones_addr - v_addr;
 #pragma unroll
   for (int kk = 0; kk < kDecTile / 16; ++kk) {
@@ -293,6 +297,7 @@ __global__ void __launch_bounds__(kF8 ? kDecThreads8 : kDecThreads, (kF8 && kR >
   constexpr int kStages = kF8 ? kDecStages8 : kDecStages;
   constexpr int kTileB = kF8 ? kDecKv8Bytes : kDecKvBytes;  // bytes of one staged K or V tile
   constexpr int kThreads = kF8 ? kDecThreads8 : kDecThreads;
+  constexpr int kN = kR < 16 ? 16 : kR;  // MMA N: query rows the MMAs compute
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   uint8_t* sK = smem;                                   // stages of K tiles
@@ -403,10 +408,10 @@ __global__ void __launch_bounds__(kF8 ? kDecThreads8 : kDecThreads, (kF8 && kR >
           if (!ok) break;
           tc_fence_after();
           if constexpr (kF8) {
-            dec_issue_qk_ts(tS + b * kDecRows, tmem + kDecTmemK + 32 * b, q_addr);
+            dec_issue_qk_ts<kN>(tS + b * kDecRows, tmem + kDecTmemK + 32 * b, q_addr);
             tc_commit(&ctl->s_full[b]);
           } else {
-            dec_issue_qk(tS + b * kDecRows, smem_u32(sK + s * kDecKvBytes), q_addr);
+            dec_issue_qk<kN>(tS + b * kDecRows, smem_u32(sK + s * kDecKvBytes), q_addr);
             tc_commit(&ctl->s_full[b]);
             tc_commit(&ctl->k_empty[s]);
           }
@@ -420,7 +425,7 @@ __global__ void __launch_bounds__(kF8 ? kDecThreads8 : kDecThreads, (kF8 && kR >
                     : mbar_wait(&ctl->v_full[s], (j / kStages) & 1, abort, &g_device_error, kDevErrTimeoutMma));
           if (!ok) break;
           tc_fence_after();
-          dec_issue_pv<kF8>(tO, kF8 ? smem_u32(sVb + (j & 1) * kDecKvBytes) : smem_u32(sV + s * kDecKvBytes),
+          dec_issue_pv<kF8, kN>(tO, kF8 ? smem_u32(sVb + (j & 1) * kDecKvBytes) : smem_u32(sV + s * kDecKvBytes),
                             ones_addr, p_addr, j > 0);
           tc_commit(&ctl->pv_done[j & 1]);
           if constexpr (!kF8) tc_commit(&ctl->v_empty[s]);
