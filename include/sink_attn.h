@@ -240,6 +240,18 @@ const char* sink_attn_status_string(sink_attn_status s);
  * entry point that synchronises. */
 int sink_attn_device_error(void* stream);
 
+/* Self-test of the bounded device waits (failure detection without a fault):
+ * one block waits on mbarriers that nothing completes.  One thread gives up
+ * after limit_ns (0 < limit_ns <= 1 s), records error code 0x107 and raises
+ * the block's abort flag; a thread of another warp, waiting with ten times
+ * that limit, must leave through the flag without recording its own code
+ * (0x108).  `out`: device pointer to 4 ints (4-byte aligned), written as
+ * {first wait returned true, its microseconds, second wait returned true,
+ * its microseconds}.  Asynchronous on `stream`; read the recorded code with
+ * sink_attn_device_error().  Returns SINK_ATTN_ERR_ALIGN for a NULL or
+ * misaligned `out`, SINK_ATTN_ERR_SHAPE for a limit outside the range. */
+sink_attn_status sink_attn_selftest_wait(unsigned long long limit_ns, int* out, void* stream);
+
 /* Profiling aid.  Registers two CUDA events (cudaEvent_t passed as void*)
  * that later calls record on their stream immediately before and after one
  * kernel launch: which = 0 -> the forward kernel of sink_attn_fwd,

@@ -18,6 +18,8 @@ enum DeviceError : int {
   kDevErrTimeoutEpilogue = 0x104,
   kDevErrTimeoutBwd = 0x105,
   kDevErrTimeoutDecode = 0x106,
+  kDevErrTimeoutSelfTest = 0x107,     // sink_attn_selftest_wait: the wait meant to give up
+  kDevErrTimeoutSelfTestAbort = 0x108,  // ... and the one meant to leave through the abort flag
   // A decode query needs a key whose cache slot already holds a newer
   // token (the ring is smaller than window + new tokens - 1).
   kDevErrDecodeCacheTooSmall = 0x201,
@@ -86,22 +88,28 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t pari
 constexpr uint32_t kWaitSleepNs = 20000;
 
 // Waits for the phase with the given parity to complete.  Gives up after
-// kWaitLimitNs, or as soon as another thread of the CTA has given up
-// (*abort != 0); on giving up it records `code` in *err (first error wins)
-// and raises *abort.  Returns true when the phase completed.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort, int* err,
-                                          int code) {
+// limit_ns, or as soon as another thread of the CTA has given up
+// (*abort != 0); on running out of time it records `code` in *err (first
+// error wins) and raises *abort.  Returns true when the phase completed.
+__device__ __forceinline__ bool mbar_wait_for(uint64_t* bar, uint32_t parity, volatile int* abort, int* err,
+                                              int code, uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   while (true) {
     if (mbar_try_wait_sleep(bar, parity, kWaitSleepNs)) return true;
     if (*abort) return false;
-    if (global_timer_ns() - t0 > kWaitLimitNs) {
+    if (global_timer_ns() - t0 > limit_ns) {
       atomicCAS(err, 0, code);
       *abort = 1;
       return false;
     }
   }
+}
+
+// mbar_wait_for with the kernels' limit, kWaitLimitNs.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort, int* err,
+                                          int code) {
+  return mbar_wait_for(bar, parity, abort, err, code, kWaitLimitNs);
 }
 
 // ----------------------------------------------------------------------- TMA

@@ -153,6 +153,35 @@ sink_attn_status plan_decode(const sink_attn_decode_dims* d, int window, float s
 }
 
 }  // namespace
+
+// Self-test of the bounded waits every kernel uses, on an mbarrier that
+// nothing ever completes.  Thread 0 gives up after limit_ns and raises the
+// CTA's abort flag; thread 32 (another warp) waits with ten times that limit
+// and must leave through the flag.  out[0], out[2]: 1 if the wait returned
+// true (neither should); out[1], out[3]: microseconds each waited.
+__global__ void __launch_bounds__(64) sink_attn_selftest_wait_kernel(unsigned long long limit_ns, int* out) {
+  __shared__ uint64_t bar[2];
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar[0], 1);
+    mbar_init(&bar[1], 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  volatile int* abort = &abort_flag;
+  if (threadIdx.x == 0 || threadIdx.x == 32) {
+    const bool first = threadIdx.x == 0;
+    const uint64_t t0 = global_timer_ns();
+    const bool ok = first ? mbar_wait_for(&bar[0], 0, abort, &g_device_error, kDevErrTimeoutSelfTest, limit_ns)
+                          : mbar_wait_for(&bar[1], 0, abort, &g_device_error, kDevErrTimeoutSelfTestAbort,
+                                          10ull * limit_ns);
+    const uint64_t us = (global_timer_ns() - t0) / 1000ull;
+    out[first ? 0 : 2] = ok ? 1 : 0;
+    out[first ? 1 : 3] = static_cast<int>(us < 0x7fffffffull ? us : 0x7fffffffull);
+  }
+}
+
 }  // namespace sa
 
 using namespace sa;
@@ -178,6 +207,13 @@ sink_attn_status sink_attn_profile_events(int which, void* ev_begin, void* ev_en
   g_profile_events[which][0] = static_cast<cudaEvent_t>(ev_begin);
   g_profile_events[which][1] = static_cast<cudaEvent_t>(ev_end);
   return SINK_ATTN_OK;
+}
+
+sink_attn_status sink_attn_selftest_wait(unsigned long long limit_ns, int* out, void* stream) {
+  if (out == nullptr || (reinterpret_cast<uintptr_t>(out) & 3u) != 0) return SINK_ATTN_ERR_ALIGN;
+  if (limit_ns == 0 || limit_ns > kWaitLimitNs) return SINK_ATTN_ERR_SHAPE;
+  sink_attn_selftest_wait_kernel<<<1, 64, 0, static_cast<cudaStream_t>(stream)>>>(limit_ns, out);
+  return cudaGetLastError() == cudaSuccess ? SINK_ATTN_OK : SINK_ATTN_ERR_CUDA;
 }
 
 int sink_attn_device_error(void* stream) {

@@ -28,7 +28,7 @@ STATUS = {
 EXPORTS = ("sink_attn_fwd", "sink_attn_bwd", "sink_attn_bwd_workspace_size", "sink_attn_status_string",
            "sink_attn_device_error", "sink_attn_fwd_launches", "sink_attn_bwd_launches", "sink_attn_profile_events",
            "sink_attn_decode", "sink_attn_decode_workspace_size", "sink_attn_decode_launches",
-           "sink_attn_decode_e4m3")
+           "sink_attn_decode_e4m3", "sink_attn_selftest_wait")
 
 
 class SinkAttnError(RuntimeError):
@@ -89,6 +89,8 @@ def load():
         L.sink_attn_decode_workspace_size.restype = ctypes.c_size_t
         L.sink_attn_decode_launches.argtypes = [DD]
         L.sink_attn_decode_launches.restype = I
+        L.sink_attn_selftest_wait.argtypes = [ctypes.c_ulonglong, P, P]
+        L.sink_attn_selftest_wait.restype = I
         _lib = L
     return _lib
 
@@ -250,6 +252,21 @@ def decode_e4m3(q, k_new, v_new, k_cache, v_cache, cache_seqlens, k_scale, v_sca
 
 def device_error(stream=None) -> int:
     return int(load().sink_attn_device_error(_stream_handle(stream)))
+
+
+def selftest_wait(limit_ns: int, out=None, stream=None):
+    """sink_attn_selftest_wait: one block waits on mbarriers nothing completes
+    (see the header).  Returns ({first returned true, its us, second returned
+    true, its us}, recorded device error code); synchronises through
+    device_error()."""
+    import torch
+    if out is None:
+        out = torch.full((4,), -1, dtype=torch.int32, device="cuda")
+    st = load().sink_attn_selftest_wait(int(limit_ns), _ptr(out), _stream_handle(stream))
+    if st != 0:
+        raise SinkAttnError(st, "sink_attn_selftest_wait")
+    code = device_error(stream)
+    return [int(v) for v in out.cpu().tolist()], code
 
 
 def fwd_launches(T, Hq, Hkv, D, batch, max_seqlen) -> int:
