@@ -338,20 +338,25 @@ def run_ours(args, rank, world, torch, dist):
     q, k, v, dout = to_dev(a["q"]), to_dev(a["k"]), to_dev(a["v"]), to_dev(a["dout"])
     sinks = torch.from_numpy(a["sinks"]).cuda()
     T = B * S
-    outs = {W: (torch.empty_like(q), torch.empty((HQ, T), dtype=torch.float32, device="cuda")) for W in LAYERS}
-    grads = {W: (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v),
-                 torch.empty((HQ,), dtype=torch.float32, device="cuda")) for W in LAYERS}
+    def out_buffers():
+        outs = {W: (torch.empty_like(q), torch.empty((HQ, T), dtype=torch.float32, device="cuda")) for W in LAYERS}
+        grads = {W: (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v),
+                     torch.empty((HQ,), dtype=torch.float32, device="cuda")) for W in LAYERS}
+        return outs, grads
+
+    outs, grads = out_buffers()
     ws = torch.empty((ops.bwd_workspace_size(T, HQ, HKV, D, B, S),), dtype=torch.uint8, device="cuda")
     stream = torch.cuda.current_stream()
-    kw = dict(batch=B, max_seqlen=S, stream=stream)
 
-    def step(q, k, v, sinks, dout, prof=None):
+    def step(q, k, v, sinks, dout, prof=None, bufs=None, st=None):
+        o_set, g_set = bufs if bufs is not None else (outs, grads)
+        kw = dict(batch=B, max_seqlen=S, stream=st if st is not None else stream)
         for W in LAYERS:
-            o, l = outs[W]
+            o, l = o_set[W]
             ops.fwd(q, k, v, sinks, None, W, 0.125, out=o, lse=l, **kw)
         for W in LAYERS:
-            o, l = outs[W]
-            dq, dk, dv, ds = grads[W]
+            o, l = o_set[W]
+            dq, dk, dv, ds = g_set[W]
             if prof is not None and W == 0:
                 ops.profile_events(ops.PROFILE_BWD_MAIN, *prof)
             ops.bwd(q, k, v, sinks, o, l, dout, None, W, 0.125, dq=dq, dk=dk, dv=dv, dsinks=ds, workspace=ws, **kw)
@@ -393,26 +398,55 @@ def run_ours(args, rank, world, torch, dist):
     value = job_throughput(world, flops, args.steps, ms)
     launches = args.steps * len(LAYERS) * (ops.fwd_launches(T, HQ, HKV, D, B, S) + ops.bwd_launches(T, HQ, HKV, D, B, S))
 
-    # ---- end to end through host buffers (pinned), copies inside the region
+    # ---- end to end through host buffers (pinned), copies inside the region.
+    # Every step copies its inputs in from pinned host memory and all of its
+    # results (outputs, lse, dq, dk, dv, dsinks of both layers) back out.  The
+    # loop is pipelined the way a caller streaming batches would write it:
+    # host-to-device copies, the step and device-to-host copies run on three
+    # streams over two sets of device buffers, so step i+1's inputs and step
+    # i-1's results cross PCIe (both directions at once) while step i runs.
     e2e_steps = max(1, min(args.steps, args.e2e_steps))
-    h_in = {n: t.cpu().pin_memory() for n, t in (("q", q), ("k", k), ("v", v), ("dout", dout), ("sinks", sinks))}
-    h_out = [t.cpu().pin_memory() for W in LAYERS for t in (*outs[W], *grads[W])]
-    d_out = [t for W in LAYERS for t in (*outs[W], *grads[W])]
+    names = ("q", "k", "v", "sinks", "dout")
+    h_in = {n: t.cpu().pin_memory() for n, t in zip(names, (q, k, v, sinks, dout))}
+    d_in = [dict(zip(names, (q, k, v, sinks, dout)))]
+    d_in.append({n: torch.empty_like(t) for n, t in d_in[0].items()})  # device copies of the device tensors
+    d_sets = [(outs, grads), out_buffers()]
+    flat = lambda bs: [t for W in LAYERS for t in (*bs[0][W], *bs[1][W])]  # noqa: E731
+    h_out = [t.cpu().pin_memory() for t in flat(d_sets[0])]
     h2d = sum(t.numel() * t.element_size() for t in h_in.values())
     d2h = sum(t.numel() * t.element_size() for t in h_out)
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    ev = lambda: torch.cuda.Event()  # noqa: E731
+    in_ready, in_free = [ev(), ev()], [ev(), ev()]
+    done, out_free = [ev(), ev()], [ev(), ev()]
     barrier()
     torch.cuda.synchronize()
     x0, x1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     x0.record(stream)
-    for _ in range(e2e_steps):
-        q.copy_(h_in["q"], non_blocking=True)
-        k.copy_(h_in["k"], non_blocking=True)
-        v.copy_(h_in["v"], non_blocking=True)
-        dout.copy_(h_in["dout"], non_blocking=True)
-        sinks.copy_(h_in["sinks"], non_blocking=True)
-        step(q, k, v, sinks, dout)
-        for h, d in zip(h_out, d_out):
-            h.copy_(d, non_blocking=True)
+    s_in.wait_event(x0)
+    s_out.wait_event(x0)
+    for i in range(e2e_steps):
+        j = i & 1
+        with torch.cuda.stream(s_in):
+            if i >= 2:
+                s_in.wait_event(in_free[j])  # step i-2 has finished reading these inputs
+            for n in names:
+                d_in[j][n].copy_(h_in[n], non_blocking=True)
+            in_ready[j].record(s_in)
+        stream.wait_event(in_ready[j])
+        if i >= 2:
+            stream.wait_event(out_free[j])  # step i-2's results have been copied out
+        dj = d_in[j]
+        step(dj["q"], dj["k"], dj["v"], dj["sinks"], dj["dout"], bufs=d_sets[j], st=stream)
+        in_free[j].record(stream)
+        done[j].record(stream)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(done[j])
+            for h, d in zip(h_out, flat(d_sets[j])):
+                h.copy_(d, non_blocking=True)
+            out_free[j].record(s_out)
+    stream.wait_event(out_free[(e2e_steps - 1) & 1])
+    stream.wait_event(in_ready[(e2e_steps - 1) & 1])
     x1.record(stream)
     torch.cuda.synchronize()
     barrier()

@@ -104,7 +104,14 @@ def make_dims(T, Hq, Hkv, D, batch, max_seqlen) -> Dims:
 
 
 def _ptr(t):
-    return None if t is None else ctypes.c_void_p(t.data_ptr())
+    """Device address of a CUDA tensor (None for None).  Every pointer of the C
+    ABI is a device pointer; a host tensor here is refused, since its address
+    would reach the kernels as if it were device memory."""
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError(f"expected a CUDA tensor, got one on {t.device}")
+    return ctypes.c_void_p(t.data_ptr())
 
 
 def _stream_handle(stream):

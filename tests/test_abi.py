@@ -154,3 +154,14 @@ def test_decode_empty_batch_is_noop(L):
     assert call_decode(L, ddims(B=0), [None] * 7, ws=None, ws_bytes=0) == 0
     assert ops.decode_launches(0, 1, 256, 257, 64, 8) == 0
     assert ops.decode_launches(4, 1, 256, 257, 64, 8) == 3
+
+
+def test_binding_refuses_host_tensors():
+    """The binding passes device pointers only: a host tensor is refused
+    before any call into the library (its address would otherwise reach the
+    kernels as device memory)."""
+    import torch
+    from sink_sliding_window_b200 import ops
+    with pytest.raises(ValueError):
+        ops._ptr(torch.zeros(4))
+    assert ops._ptr(None) is None
