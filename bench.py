@@ -265,6 +265,50 @@ def measure_decode(torch, ops, stream, iters=20):
     return res
 
 
+def measure_layers(torch, ops, stream, q, k, v, sinks, dout, outs, grads, ws, iters=20):
+    """Forward and backward of each layer alone (CUDA events on the launching
+    stream, mean over `iters` calls after 3 warm-up calls): TFLOP/s on the
+    counted pairs, and GB/s of the layer's minimum DRAM bytes (every input
+    read once, every output written once) against the measured HBM peak; the
+    window-128 layers are judged on the latter.  q, dout, out and dq (134 MB
+    each) exceed the 126 MB L2, so no flush between calls."""
+    _, hbm, kind = read_peaks()
+    nb = lambda *ts: sum(t.numel() * t.element_size() for t in ts)  # noqa: E731
+    res = []
+    for W in LAYERS:
+        o, l = outs[W]
+        dq, dk, dv, ds = grads[W]
+        kw = dict(batch=B, max_seqlen=S, stream=stream)
+        calls = {
+            "fwd": (lambda: ops.fwd(q, k, v, sinks, None, W, 0.125, out=o, lse=l, **kw),
+                    nb(q, k, v, sinks) + nb(o, l)),
+            "bwd": (lambda: ops.bwd(q, k, v, sinks, o, l, dout, None, W, 0.125, dq=dq, dk=dk, dv=dv, dsinks=ds,
+                                    workspace=ws, **kw),
+                    nb(q, k, v, sinks, o, l, dout) + nb(dq, dk, dv, ds)),
+        }
+        fl = dict(zip(("fwd", "bwd"), layer_flops(W)))
+        entry = {"window": W, "workload": f"{WORKLOAD} ({'window %d' % W if W > 0 else 'full causal'})"}
+        for name, (fn, min_bytes) in calls.items():
+            for _ in range(3):
+                fn()
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(iters):
+                fn()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            ms = e0.elapsed_time(e1) / iters
+            entry[name] = {"ms": ms, "tflops": fl[name] / ms / 1e9, "min_bytes": min_bytes,
+                           "GBps": min_bytes / ms / 1e6, "hbm_frac": min_bytes / ms / 1e6 / hbm}
+        entry["peak_GBps"] = hbm
+        entry["peak_source"] = f"{kind} hbm_gbs"
+        res.append(entry)
+    if ops.device_error() != 0:
+        raise RuntimeError("a kernel reported a timed-out wait")
+    return res
+
+
 # ----------------------------------------------------------- aggregation
 def max_over_ranks(x, dist, device):
     """Largest value of x over all ranks (the slowest rank's time); x itself
@@ -453,6 +497,7 @@ def run_ours(args, rank, world, torch, dist):
     e2e_ms = max_over_ranks(x0.elapsed_time(x1), dist, "cuda")
     e2e_value = job_throughput(world, flops, e2e_steps, e2e_ms)
 
+    layers = measure_layers(torch, ops, stream, q, k, v, sinks, dout, outs, grads, ws)
     decode = measure_decode(torch, ops, stream) if not args.skip_decode else None
 
     if rank != 0:
@@ -475,6 +520,7 @@ def run_ours(args, rank, world, torch, dist):
         "gpu_launches": launches,
         "clocks": clk,
     }
+    line["layers"] = layers
     if decode is not None:
         line["decode"] = decode
     if world == 1 and not args.skip_cpu_baseline:
