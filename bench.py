@@ -220,12 +220,15 @@ def measure_decode(torch, ops, stream, iters=20):
         mk = lambda *shape: torch.randn(*shape, device="cuda", generator=g).to(torch.bfloat16)  # noqa: E731
         q, kn, vn = mk(Bd, Lq, HQ, D), mk(Bd, Lq, HKV, D), mk(Bd, Lq, HKV, D)
         if f8:
-            # e4m3 codes of both signs, NaN codes (0x7F, 0xFF) excluded; one scale per KV head
-            codes = lambda: (torch.randint(0, 0x7F, (Bd, C, HKV, D), dtype=torch.uint8, device="cuda", generator=g)  # noqa: E731
-                             | (torch.randint(0, 2, (Bd, C, HKV, D), dtype=torch.uint8, device="cuda", generator=g) << 7))
-            kc, vc = codes(), codes()
-            k_scale = torch.full((HKV,), 1.0 / 64, dtype=torch.float32, device="cuda")
-            v_scale = torch.full((HKV,), 1.0 / 64, dtype=torch.float32, device="cuda")
+            # The N(0,1) bf16 history quantised to e4m3 with one scale per KV
+            # head (amax / 448), as an FP8 cache would hold it (input preparation
+            # only; the timed call reads the codes).
+            def quantised():
+                x = mk(Bd, C, HKV, D).float()
+                sc = x.abs().amax(dim=(0, 1, 3)) / 448.0
+                return (x / sc[None, None, :, None]).to(torch.float8_e4m3fn).view(torch.uint8), sc
+            kc, k_scale = quantised()
+            vc, v_scale = quantised()
         else:
             kc, vc = mk(Bd, C, HKV, D), mk(Bd, C, HKV, D)
         sl = torch.full((Bd,), L0, dtype=torch.int32, device="cuda")
