@@ -153,11 +153,14 @@ def test_launch_count(ops):
 
 
 # ----------------------------------------------------------------- e4m3 cache
-def _run_e4m3(ops, cached, Lq, Hq, Hkv, C, window, seed, seqs=None):
+def _run_e4m3(ops, cached, Lq, Hq, Hkv, C, window, seed, seqs=None, heavy=False):
     """The e4m3-cache decode: history tokens enter the cache as host-quantised
     codes (per-head scale = amax / 448), the new tokens are quantised by the
     call.  The oracle gets the dequantised values code * scale exactly (fp64),
-    so the comparison measures the kernel, not the quantisation."""
+    so the comparison measures the kernel, not the quantisation.  heavy: the
+    history slots instead hold codes drawn uniformly over every finite e4m3
+    code of both signs (scale 1/64): heavy-tailed logits, so the running
+    reference max of a row is raised on many tiles, not just the first."""
     import torch
     from tests import e4m3
     a = synth.decode_inputs(seed, cached, Lq, Hq, Hkv)
@@ -165,10 +168,20 @@ def _run_e4m3(ops, cached, Lq, Hq, Hkv, C, window, seed, seqs=None):
     B = len(cached)
     kf = synth.bf16_bits_to_f32(a["k"])
     vf = synth.bf16_bits_to_f32(a["v"])
-    ks = (np.abs(kf).max(axis=(0, 2)) / np.float32(448.0)).astype(np.float32)
-    vs = (np.abs(vf).max(axis=(0, 2)) / np.float32(448.0)).astype(np.float32)
+    if heavy:
+        ks = np.full(Hkv, 1.0 / 64.0, np.float32)
+        vs = np.full(Hkv, 1.0 / 64.0, np.float32)
+    else:
+        ks = (np.abs(kf).max(axis=(0, 2)) / np.float32(448.0)).astype(np.float32)
+        vs = (np.abs(vf).max(axis=(0, 2)) / np.float32(448.0)).astype(np.float32)
     ck = e4m3.quantize(kf * (np.float32(1.0) / ks)[None, :, None])
     cv = e4m3.quantize(vf * (np.float32(1.0) / vs)[None, :, None])
+    if heavy:
+        rng = np.random.default_rng(seed)
+        hist = np.concatenate([np.arange(int(cu[b]), int(cu[b]) + int(cached[b])) for b in range(B)]).astype(np.int64)
+        for c in (ck, cv):
+            shape = (len(hist), Hkv, 64)
+            c[hist] = (rng.integers(0, 0x7F, size=shape) | (rng.integers(0, 2, size=shape) << 7)).astype(np.uint8)
     kc0 = np.full((B, C, Hkv, 64), 0x7F, np.uint8)  # unused slots hold the NaN code
     vc0 = np.full((B, C, Hkv, 64), 0x7F, np.uint8)
     for b in range(B):
@@ -220,6 +233,13 @@ def test_e4m3_cache(ops, window, C, Lq):
 @pytest.mark.parametrize("G,Lq", [(8, 4), (16, 4)])
 def test_e4m3_cache_row_variants(ops, G, Lq):
     _run_e4m3(ops, [0, 64, 257], Lq, 2 * G, 2, 512, 0, seed=70 + G)
+
+
+@pytest.mark.parametrize("window", [0, 100])
+def test_e4m3_cache_heavy_tailed(ops, window):
+    """Many reference-max raises per CTA in the e4m3 variant (each one a CTA
+    vote, an exact tile max and a rescale of O)."""
+    _run_e4m3(ops, [1000, 2000, 4095, 3], 1, 16, 2, 4096, window, seed=90 + window, heavy=True)
 
 
 def test_e4m3_cache_gpt_oss_full_size(ops):
