@@ -32,8 +32,8 @@ def test_tiny_whole(ops, name):
     check(host_f64(lse), rl, TOL_LSE, f"{name} lse")
 
 
-def _small(T, Hq, Hkv, cu, window, seed, sinks=None):
-    w = synth.Workload("edge", T, Hq, Hkv, 64, np.asarray(cu, np.int32), None, window, 0.125, seed=seed)
+def _small(T, Hq, Hkv, cu, window, seed, sinks=None, scale=0.125):
+    w = synth.Workload("edge", T, Hq, Hkv, 64, np.asarray(cu, np.int32), None, window, scale, seed=seed)
     a = w.generate()
     if sinks is not None:
         a["sinks"] = np.asarray(sinks, np.float32)
@@ -60,6 +60,15 @@ def test_gqa_ratios(ops, G):
     Hkv = 2
     w, a = _small(400, G * Hkv, Hkv, [0, 37, 38, 400], 100, seed=G)
     _whole_check(ops, w, a, f"G={G}")
+
+
+@pytest.mark.parametrize("scale", [1.0, 4.0])
+@pytest.mark.parametrize("window", [0, 64])
+def test_wide_logits(ops, scale, window):
+    """Logits 8-32x wider than at scale 1/8: a row's running reference max is
+    raised on many key steps, so the O rescale runs repeatedly."""
+    w, a = _small(700, 8, 1, [0, 250, 700], window, seed=11, scale=scale)
+    _whole_check(ops, w, a, f"scale={scale} W={window}")
 
 
 def test_sink_extremes(ops):
