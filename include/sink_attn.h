@@ -50,7 +50,8 @@
  *     <= 128; scale finite and > 0; bf16 tensors 16-byte aligned.
  *   - A device-side wait that exceeds its time limit (about one second; it
  *     never happens in a correct build) makes the kernel record an error
- *     code and return instead of hanging; sink_attn_device_error() reads it.
+ *     code and return instead of hanging; sink_attn_last_device_error()
+ *     reads it.
  */
 #ifndef SINK_ATTN_H_
 #define SINK_ATTN_H_
@@ -68,7 +69,7 @@ typedef enum {
     SINK_ATTN_ERR_ALIGN = 3,         /* a tensor is not 16-byte aligned */
     SINK_ATTN_ERR_UNSUPPORTED = 4,   /* valid, but outside what this build implements */
     SINK_ATTN_ERR_CUDA = 5,          /* a CUDA runtime/driver call failed */
-    SINK_ATTN_ERR_DEVICE_TIMEOUT = 6,/* a kernel gave up on a wait (see sink_attn_device_error) */
+    SINK_ATTN_ERR_DEVICE_TIMEOUT = 6,/* a kernel gave up on a wait (see sink_attn_last_device_error) */
     SINK_ATTN_ERR_WORKSPACE = 7      /* workspace missing or smaller than sink_attn_bwd_workspace_size() */
 } sink_attn_status;
 
@@ -101,10 +102,11 @@ size_t sink_attn_bwd_workspace_size(const sink_attn_dims* dims);
  * and the upstream gradient dout [T][Hq][D] bf16.  Writes (overwrites, does
  * not accumulate) dq [T][Hq][D], dk, dv [T][Hkv][D] (bf16) and dsinks [Hq]
  * (fp32).  dsinks is reduced in a fixed order and is bitwise reproducible
- * run to run; dq is accumulated with fp32 atomics and may differ in the last
- * bits between runs.  `workspace` is caller-owned device memory of at least
- * sink_attn_bwd_workspace_size(dims) bytes, 256-byte aligned; its contents on
- * entry do not matter. */
+ * run to run; dq is summed over key tiles in an fp32 accumulator by TMA
+ * bulk reduce-adds (performed in L2 in whatever order the tiles finish), so
+ * it may differ in the last bits between runs.  `workspace` is caller-owned
+ * device memory of at least sink_attn_bwd_workspace_size(dims) bytes,
+ * 256-byte aligned; its contents on entry do not matter. */
 sink_attn_status sink_attn_bwd(const sink_attn_dims* dims,
                                const void* q, const void* k, const void* v,
                                const float* sinks, const int* cu_seqlens,
@@ -215,8 +217,11 @@ sink_attn_status sink_attn_decode(const sink_attn_decode_dims* dims,
  * fp32 [Hkv], device, > 0).  The pages list FP8 training recipes (Megatron-LM
  * issue 1739 and its example scripts); this is the place on this path where
  * FP8 pays on B200 at head dim 64: decode is HBM-bound, and e4m3 storage
- * halves the bytes the cache moves, while the MMAs stay bf16 (e4m3 values
- * are exact in bf16).  The call quantises the new tokens' k_new / v_new
+ * halves the bytes the cache moves.  The kernel widens the codes to fp16
+ * (every e4m3 value is exact in fp16) and runs fp16 MMAs, so the queries are
+ * converted from bf16 to fp16 for them: a query element beyond the fp16
+ * range saturates to +-65504, the one input-range limit of this variant
+ * (sink_attn_decode has none).  The call quantises the new tokens' k_new / v_new
  * (bf16) as code = e4m3(x * (1 / scale)), rounded to nearest even and
  * saturated to +-448, into their slots.  The workspace size is that of
  * sink_attn_decode_workspace_size(). */
@@ -235,9 +240,13 @@ int sink_attn_decode_launches(const sink_attn_decode_dims* dims);
 /* Human-readable name of a status code (static string, never NULL). */
 const char* sink_attn_status_string(sink_attn_status s);
 
-/* Synchronises `stream`, then returns and clears the device error code that a
- * timed-out wait recorded on the current device (0 = none).  This is the only
- * entry point that synchronises. */
+/* Synchronises `stream` (a cudaStream_t passed as void*), then returns and
+ * clears the device error code that a timed-out wait (or a decode ring too
+ * small for its window) recorded on the current device: 0 = none, -1 = the
+ * synchronisation or the read failed.  These are the only entry points that
+ * synchronise.  sink_attn_device_error is the same function under a shorter
+ * name. */
+int sink_attn_last_device_error(void* stream);
 int sink_attn_device_error(void* stream);
 
 /* Self-test of the bounded device waits (failure detection without a fault):

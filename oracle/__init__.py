@@ -58,10 +58,13 @@ def _bind(path):
     lib.oracle_bwd_dq_rows_bf16.argtypes = common + [P, P, P, P, I, Dbl, P, P, P, I64, P, I]
     lib.oracle_bwd_dkv_rows_f64.argtypes = common + [P, P, P, P, I, Dbl, P, P, P, I64, P, P, I]
     lib.oracle_bwd_dkv_rows_bf16.argtypes = common + [P, P, P, P, I, Dbl, P, P, P, I64, P, P, I]
+    lib.oracle_bwd_dsinks_f64.argtypes = common + [P, P, P, P, I, Dbl, P, P, P, I]
+    lib.oracle_bwd_dsinks_bf16.argtypes = common + [P, P, P, P, I, Dbl, P, P, P, I]
     lib.oracle_bf16_to_f64.argtypes = [P, P, I64]
     for f in ("oracle_fwd_f64", "oracle_fwd_bf16", "oracle_fwd_rows_f64", "oracle_fwd_rows_bf16",
               "oracle_bwd_f64", "oracle_bwd_bf16", "oracle_bwd_dq_rows_f64", "oracle_bwd_dq_rows_bf16",
-              "oracle_bwd_dkv_rows_f64", "oracle_bwd_dkv_rows_bf16", "oracle_bf16_to_f64", "oracle_max_threads"):
+              "oracle_bwd_dkv_rows_f64", "oracle_bwd_dkv_rows_bf16", "oracle_bwd_dsinks_f64",
+              "oracle_bwd_dsinks_bf16", "oracle_bf16_to_f64", "oracle_max_threads"):
         getattr(lib, f).restype = I
     return lib
 
@@ -197,6 +200,20 @@ class Oracle:
         _check(rc, "oracle bwd_dkv_rows")
         return dk, dv
 
+    def bwd_dsinks(self, q, k, v, sinks, cu_seqlens, window, scale, dout, out_for_D=None, nthreads=0):
+        """dsinks of the backward definition alone (one forward pass of
+        work).  Returns dsinks [Hq] float64."""
+        T, Hq, D = q.shape
+        Hkv = k.shape[1]
+        cu = _cu(cu_seqlens, T)
+        ds = np.empty((Hq,), np.float64)
+        args, s, o, do, sfx = self._bwd_args(q, k, v, sinks, dout, out_for_D)
+        fn = getattr(self.lib, f"oracle_bwd_dsinks_{sfx}")
+        rc = fn(T, Hq, Hkv, D, cu.shape[0] - 1, _ptr(cu), *map(_ptr, args), _ptr(s), int(window), float(scale),
+                _ptr(o), _ptr(do), _ptr(ds), int(nthreads))
+        _check(rc, "oracle bwd_dsinks")
+        return ds
+
     def bf16_bits_to_f64(self, a):
         """Exact widening of bf16 bit patterns (uint16) to float64."""
         a = np.ascontiguousarray(a, np.uint16)
@@ -254,6 +271,10 @@ def bwd_dq_rows(*a, **kw):
 
 def bwd_dkv_rows(*a, **kw):
     return default().bwd_dkv_rows(*a, **kw)
+
+
+def bwd_dsinks(*a, **kw):
+    return default().bwd_dsinks(*a, **kw)
 
 
 def bf16_bits_to_f64(a):

@@ -296,6 +296,61 @@ int oracle_bwd_f64(int T, int Hq, int Hkv, int D, int B, const int32_t* cu_seqle
     return err;
 }
 
+/* The sink gradient alone, fp64 inputs:
+ *   dsinks_h = -sum over every document and query token i of P_sink,i D_i,
+ *   P_sink,i = exp(s_h - lse_i),  D_i = dout_i . out_i.
+ * It needs each row's lse and output only, i.e. one forward pass, not the
+ * whole backward.  out_for_D as for oracle_bwd_f64.  Each row's term is
+ * formed independently; each head then sums its terms in ascending token
+ * order. */
+int oracle_bwd_dsinks_f64(int T, int Hq, int Hkv, int D, int B, const int32_t* cu_seqlens,
+                          const double* q, const double* k, const double* v, const double* sinks,
+                          int window, double scale, const double* out_for_D, const double* dout,
+                          double* dsinks, int nthreads) {
+    if (!check_common(T, Hq, Hkv, D, B, cu_seqlens) || !sinks || !dsinks) return ORACLE_ERR_ARG;
+    if (T > 0 && (!q || !k || !v || !dout)) return ORACLE_ERR_ARG;
+    int64_t maxlen = 0;
+    for (int b = 0; b < B; ++b)
+        if (cu_seqlens[b + 1] - cu_seqlens[b] > maxlen) maxlen = cu_seqlens[b + 1] - cu_seqlens[b];
+    double* term = (double*)malloc(sizeof(double) * (size_t)(T > 0 ? T : 1) * Hq);
+    if (!term) return ORACLE_ERR_NOMEM;
+    int err = ORACLE_OK;
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#endif
+#pragma omp parallel
+    {
+        double* logits = (double*)malloc(sizeof(double) * (size_t)(maxlen > 0 ? maxlen : 1));
+        double* orow = (double*)malloc(sizeof(double) * (size_t)D);
+        if (!logits || !orow) {
+#pragma omp atomic write
+            err = ORACLE_ERR_NOMEM;
+        } else {
+#pragma omp for schedule(dynamic, 16)
+            for (int64_t row = 0; row < (int64_t)T * Hq; ++row) {
+                int64_t t = row / Hq;
+                int h = (int)(row % Hq);
+                int64_t a = cu_seqlens[doc_of(cu_seqlens, B, t)];
+                double lse = fwd_row(t, h, a, Hq, Hkv, D, q, k, v, sinks[h], window, scale, logits, orow);
+                const double* o = out_for_D ? out_for_D + (t * Hq + h) * (int64_t)D : orow;
+                const double* doi = dout + (t * Hq + h) * (int64_t)D;
+                double Di = 0.0;
+                for (int d = 0; d < D; ++d) Di += doi[d] * o[d];
+                term[(int64_t)h * T + t] = exp(sinks[h] - lse) * Di;
+            }
+        }
+        free(logits);
+        free(orow);
+    }
+    for (int h = 0; h < Hq; ++h) {
+        double acc = 0.0;
+        for (int64_t t = 0; t < T; ++t) acc -= term[(int64_t)h * T + t];
+        dsinks[h] = acc;
+    }
+    free(term);
+    return err;
+}
+
 /* Backward restricted to chosen query tokens: dq for every head of each
  * token in `rows` (fp64 inputs).  dq_i only needs row i's own probabilities,
  * so each row is the definition above evaluated for that row alone.
@@ -522,6 +577,26 @@ int oracle_bwd_bf16(int T, int Hq, int Hkv, int D, int B, const int32_t* cu_seql
     if (qd && kd && vd && dod && sd && (od || !out_for_D_bf16))
         rc = oracle_bwd_f64(T, Hq, Hkv, D, B, cu_seqlens, qd, kd, vd, sd, window, scale, od, dod, dq, dk, dv,
                             dsinks, nthreads);
+    free(qd); free(kd); free(vd); free(dod); free(od); free(sd);
+    return rc;
+}
+
+int oracle_bwd_dsinks_bf16(int T, int Hq, int Hkv, int D, int B, const int32_t* cu_seqlens,
+                           const uint16_t* q, const uint16_t* k, const uint16_t* v, const float* sinks,
+                           int window, double scale, const uint16_t* out_for_D_bf16, const uint16_t* dout,
+                           double* dsinks, int nthreads) {
+    if (T < 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || !sinks) return ORACLE_ERR_ARG;
+    if (T > 0 && (!q || !k || !v || !dout)) return ORACLE_ERR_ARG;
+    double* qd = widen(q, (int64_t)T * Hq * D);
+    double* kd = widen(k, (int64_t)T * Hkv * D);
+    double* vd = widen(v, (int64_t)T * Hkv * D);
+    double* dod = widen(dout, (int64_t)T * Hq * D);
+    double* od = out_for_D_bf16 ? widen(out_for_D_bf16, (int64_t)T * Hq * D) : NULL;
+    double* sd = widen_f32(sinks, Hq);
+    int rc = ORACLE_ERR_NOMEM;
+    if (qd && kd && vd && dod && sd && (od || !out_for_D_bf16))
+        rc = oracle_bwd_dsinks_f64(T, Hq, Hkv, D, B, cu_seqlens, qd, kd, vd, sd, window, scale, od, dod, dsinks,
+                                   nthreads);
     free(qd); free(kd); free(vd); free(dod); free(od); free(sd);
     return rc;
 }

@@ -713,13 +713,8 @@ inline sink_attn_status bwd_launch(const Geometry& geo, float scale, const void*
       !make_map_3d(&tv, v, kHeadDim, geo.Hkv, geo.T, 1, kBlockN) ||
       !make_map_3d_f32(&tdq, dq_acc, kHeadDim, geo.Hq, geo.T, G, 1 << geo.P_log2))
     return SINK_ATTN_ERR_CUDA;
-  static int smem_set = 0;
-  if (!smem_set) {
-    if (cudaFuncSetAttribute(sink_attn_bwd_main_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(kBwdSmemBytes)) != cudaSuccess)
-      return SINK_ATTN_ERR_CUDA;
-    smem_set = 1;
-  }
+  static SmemAttrOnce smem_set;
+  if (!smem_set.ensure(sink_attn_bwd_main_kernel, kBwdSmemBytes)) return SINK_ATTN_ERR_CUDA;
   BwdParams bp;
   bp.geo = geo;
   bp.scale = scale;

@@ -67,16 +67,6 @@ sink_attn_status check_dims(const sink_attn_dims* d, const int* cu_seqlens, bool
 // Events registered by sink_attn_profile_events: [which][begin/end].
 cudaEvent_t g_profile_events[2][2] = {{nullptr, nullptr}, {nullptr, nullptr}};
 
-template <typename K>
-bool set_smem_once(K kernel, size_t bytes, int* done_flag) {
-  // Per process; the attribute is per function, not per device context.
-  if (*done_flag) return true;
-  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes)) !=
-      cudaSuccess)
-    return false;
-  *done_flag = 1;
-  return true;
-}
 
 // Decode: sizes, split count and workspace layout of one call.
 struct DecPlan {
@@ -216,7 +206,7 @@ sink_attn_status sink_attn_selftest_wait(unsigned long long limit_ns, int* out, 
   return cudaGetLastError() == cudaSuccess ? SINK_ATTN_OK : SINK_ATTN_ERR_CUDA;
 }
 
-int sink_attn_device_error(void* stream) {
+int sink_attn_last_device_error(void* stream) {
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (cudaStreamSynchronize(st) != cudaSuccess) return -1;
   int v = 0, zero = 0;
@@ -224,6 +214,8 @@ int sink_attn_device_error(void* stream) {
   if (v != 0 && cudaMemcpyToSymbol(g_device_error, &zero, sizeof(int)) != cudaSuccess) return -1;
   return v;
 }
+
+int sink_attn_device_error(void* stream) { return sink_attn_last_device_error(stream); }
 
 int sink_attn_fwd_launches(const sink_attn_dims* d) {
   Geometry geo;
@@ -251,8 +243,8 @@ sink_attn_status sink_attn_fwd(const sink_attn_dims* d, const void* q, const voi
       !make_map_3d(&tv, v, kHeadDim, geo.Hkv, geo.T, 1, kBlockN))
     return SINK_ATTN_ERR_CUDA;
 
-  static int smem_set = 0;
-  if (!set_smem_once(sink_attn_fwd_kernel, kFwdSmemBytes, &smem_set)) return SINK_ATTN_ERR_CUDA;
+  static SmemAttrOnce smem_set;
+  if (!smem_set.ensure(sink_attn_fwd_kernel, kFwdSmemBytes)) return SINK_ATTN_ERR_CUDA;
 
   FwdParams p;
   p.geo = geo;
@@ -321,7 +313,6 @@ namespace {
 
 static __device__ __align__(256) uint8_t g_noalloc_scratch[SINK_ATTN_NOALLOC_SCRATCH_BYTES];
 
-constexpr int kMaxDevices = 64;
 std::mutex g_noalloc_mutex;
 void* g_noalloc_ptr[kMaxDevices] = {};
 
@@ -419,11 +410,11 @@ sink_attn_status decode_impl(const sink_attn_decode_dims* d, const void* q, cons
        sink_attn_decode_kernel<64, false>},
       {sink_attn_decode_kernel<8, true>, sink_attn_decode_kernel<16, true>, sink_attn_decode_kernel<32, true>,
        sink_attn_decode_kernel<64, true>}};
-  static int smem_set[2][4] = {{0, 0, 0, 0}, {0, 0, 0, 0}};
+  static SmemAttrOnce smem_set[2][4];
   const int vi = p.R <= 8 ? 0 : (p.R <= 16 ? 1 : (p.R <= 32 ? 2 : 3));
   const Kern kern = kerns[e4m3][vi];
   const size_t smem = e4m3 ? kDecSmemBytes8 : kDecSmemBytes;
-  if (!set_smem_once(kern, smem, &smem_set[e4m3][vi])) return SINK_ATTN_ERR_CUDA;
+  if (!smem_set[e4m3][vi].ensure(kern, smem)) return SINK_ATTN_ERR_CUDA;
   const long long ctas = static_cast<long long>(p.batch) * p.Hkv * p.n_split;
   if (ctas > 0x7fffffff) return SINK_ATTN_ERR_UNSUPPORTED;
 

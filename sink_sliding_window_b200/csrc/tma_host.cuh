@@ -5,9 +5,34 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <mutex>
 
 namespace sa {
+
+// Devices per process the library keeps per-device state for.
+constexpr int kMaxDevices = 64;
+
+// Raises a kernel's dynamic shared-memory limit once per device.  The CUDA
+// runtime applies cudaFuncSetAttribute to the function on the current
+// device only, so a process that launches on several devices needs the call
+// on each of them.  Thread-safe: the flags are atomics, and a race between
+// two first calls on one device only repeats the (idempotent) call.
+struct SmemAttrOnce {
+  std::atomic<int> done[kMaxDevices] = {};
+
+  template <typename K>
+  bool ensure(K kernel, size_t bytes) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return false;
+    if (dev < kMaxDevices && done[dev].load(std::memory_order_acquire)) return true;
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes)) !=
+        cudaSuccess)
+      return false;
+    if (dev < kMaxDevices) done[dev].store(1, std::memory_order_release);
+    return true;
+  }
+};
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                    const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,

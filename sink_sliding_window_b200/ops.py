@@ -26,7 +26,7 @@ STATUS = {
 }
 
 EXPORTS = ("sink_attn_fwd", "sink_attn_bwd", "sink_attn_bwd_workspace_size", "sink_attn_status_string",
-           "sink_attn_device_error", "sink_attn_fwd_launches", "sink_attn_bwd_launches", "sink_attn_profile_events",
+           "sink_attn_last_device_error", "sink_attn_device_error", "sink_attn_fwd_launches", "sink_attn_bwd_launches", "sink_attn_profile_events",
            "sink_attn_decode", "sink_attn_decode_workspace_size", "sink_attn_decode_launches",
            "sink_attn_decode_e4m3", "sink_attn_selftest_wait")
 
@@ -71,6 +71,8 @@ def load():
         L.sink_attn_bwd_workspace_size.restype = ctypes.c_size_t
         L.sink_attn_status_string.argtypes = [I]
         L.sink_attn_status_string.restype = ctypes.c_char_p
+        L.sink_attn_last_device_error.argtypes = [P]
+        L.sink_attn_last_device_error.restype = I
         L.sink_attn_device_error.argtypes = [P]
         L.sink_attn_device_error.restype = I
         L.sink_attn_fwd_launches.argtypes = [DP]
@@ -258,7 +260,7 @@ def decode_e4m3(q, k_new, v_new, k_cache, v_cache, cache_seqlens, k_scale, v_sca
 
 
 def device_error(stream=None) -> int:
-    return int(load().sink_attn_device_error(_stream_handle(stream)))
+    return int(load().sink_attn_last_device_error(_stream_handle(stream)))
 
 
 def selftest_wait(limit_ns: int, out=None, stream=None):

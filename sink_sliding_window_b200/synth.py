@@ -101,9 +101,11 @@ class Workload:
         return a
 
     def sample_rows(self, n: int) -> np.ndarray:
-        """Seeded sample of query tokens: document starts and ends, the first
-        and last 130 tokens of the first document (tile edges), and random
-        tokens; sorted and unique."""
+        """Seeded sample of query tokens: for each of the first 8 documents
+        five fixed tokens (its first, second and last token, and the tokens
+        127 and 128 places after its start, which sit on either side of a
+        128-token tile edge), then random tokens up to n; sorted and
+        unique."""
         rng = _rng(self.seed, "rows")
         c = self.cu_seqlens.astype(np.int64)
         fixed = set()

@@ -357,6 +357,108 @@ def pin_restricted_backward(O):
         rk, rv = O.bwd_dkv_rows(q, k, v, s, cu, W, 0.25, dout, keys)
         assert_close(rk, dk[keys], 1e-12, f"dk rows case {n}")
         assert_close(rv, dv[keys], 1e-12, f"dv rows case {n}")
+        # the sink gradient alone equals the full backward's
+        ds = O.bwd(q, k, v, s, cu, W, 0.25, dout)[3]
+        assert_close(O.bwd_dsinks(q, k, v, s, cu, W, 0.25, dout), ds, 1e-12, f"dsinks alone case {n}")
+
+
+def _probabilities(q, k, s, cu, W, scale):
+    """P_ij = e^{l_ij - lse_i} and P_sink,i = e^{s_h - lse_i}, written out in
+    numpy from the definition (independent of the oracle): P [Hq, T, T]
+    (zero where key j is not allowed for query i) and Psink [Hq, T]."""
+    T, Hq, _ = q.shape
+    Hkv = k.shape[1]
+    G = Hq // Hkv
+    P = np.zeros((Hq, T, T))
+    Psink = np.zeros((Hq, T))
+    for b in range(len(cu) - 1):
+        a, e = int(cu[b]), int(cu[b + 1])
+        for i in range(a, e):
+            lo = a if W <= 0 else max(a, i - W + 1)
+            for h in range(Hq):
+                lg = scale * (k[lo:i + 1, h // G] @ q[i, h])
+                m = max(float(s[h]), float(lg.max()))
+                z = math.exp(float(s[h]) - m) + float(np.exp(lg - m).sum())
+                P[h, i, lo:i + 1] = np.exp(lg - m) / z
+                Psink[h, i] = math.exp(float(s[h]) - m) / z
+    return P, Psink
+
+
+def pin_saved_output_for_D(O):
+    """The backward's optional saved output (``out_for_D``, the output the
+    caller kept from its forward) enters only through D_i = dout_i . X_i:
+      (a) X = the oracle's own forward output gives exactly the results of
+          X = None, in the full backward and in both restricted ones;
+      (b) for another X, dsinks_h = -sum_i P_sink,i (dout_i . X_i);
+      (c) dv does not move, and dq, dk move by the closed-form change of
+          dS_ij by -P_ij dout_i . (X_i - out_i):
+            dq_i += -scale sum_j P_ij delta_i k_j,
+            dk_j += -scale sum_{i, h in group} P_ij delta_i q_i,
+          delta_i = dout_i . (X_i - out_i);
+      (d) the restricted backwards take X at the right rows;
+      (e) the bf16 entry point widens X exactly, like every other input."""
+    scale = 0.3
+    for n, (cu, W) in enumerate([([0, 16], 0), ([0, 16], 5), ([0, 6, 16], 0), ([0, 5, 7, 16], 3)]):
+        q, k, v, s, cu = rand_problem(140 + n, 16, 4, 2, 8, cu=cu)
+        T, Hq, D = q.shape
+        G = Hq // k.shape[1]
+        rng = np.random.default_rng(150 + n)
+        dout = rng.standard_normal(q.shape)
+        out, lse = O.fwd(q, k, v, s, cu, W, scale)
+        base = O.bwd(q, k, v, s, cu, W, scale, dout)
+        same = O.bwd(q, k, v, s, cu, W, scale, dout, out_for_D=out)
+        assert all(np.array_equal(x, y) for x, y in zip(base, same)), f"saved output = own output, case {n}"
+        rows = np.array([0, 5, 6, 11, 15])
+        assert np.array_equal(O.bwd_dq_rows(q, k, v, s, cu, W, scale, dout, rows, out_for_D=out),
+                              O.bwd_dq_rows(q, k, v, s, cu, W, scale, dout, rows)), f"dq rows own output {n}"
+        rk0, rv0 = O.bwd_dkv_rows(q, k, v, s, cu, W, scale, dout, rows)
+        rk1, rv1 = O.bwd_dkv_rows(q, k, v, s, cu, W, scale, dout, rows, out_for_D=out)
+        assert np.array_equal(rk0, rk1) and np.array_equal(rv0, rv1), f"dk/dv rows own output {n}"
+
+        X = out + 0.5 * rng.standard_normal(out.shape)
+        dq0, dk0, dv0, ds0 = base
+        dq1, dk1, dv1, ds1 = O.bwd(q, k, v, s, cu, W, scale, dout, out_for_D=X)
+        P, Psink = _probabilities(q, k, s, cu, W, scale)
+        DX = np.einsum("thd,thd->ht", dout, X)  # [Hq, T]
+        assert_close(ds1, -(Psink * DX).sum(axis=1), 1e-12, f"dsinks from saved output, case {n}")
+        assert_close(O.bwd_dsinks(q, k, v, s, cu, W, scale, dout, out_for_D=X), -(Psink * DX).sum(axis=1), 1e-12,
+                     f"dsinks alone from saved output, case {n}")
+        assert np.array_equal(dv0, dv1), f"dv must not depend on the saved output, case {n}"
+        delta = np.einsum("thd,thd->ht", dout, X - out)  # [Hq, T]
+        kk = np.repeat(k, G, axis=1)  # [T, Hq, D]: key j as seen by head h
+        ddq = -scale * np.einsum("hij,jhd->ihd", P * delta[:, :, None], kk)
+        assert_close(dq1 - dq0, ddq, 1e-12, f"dq shift from saved output, case {n}")
+        ddk_h = -scale * np.einsum("hij,ihd->jhd", P * delta[:, :, None], q)  # [T, Hq, D]
+        ddk = ddk_h.reshape(T, Hq // G, G, D).sum(axis=2)
+        assert_close(dk1 - dk0, ddk, 1e-12, f"dk shift from saved output, case {n}")
+        assert_close(O.bwd_dq_rows(q, k, v, s, cu, W, scale, dout, rows, out_for_D=X), dq1[rows], 1e-12,
+                     f"dq rows with saved output, case {n}")
+        rk, rv = O.bwd_dkv_rows(q, k, v, s, cu, W, scale, dout, rows, out_for_D=X)
+        assert_close(rk, dk1[rows], 1e-12, f"dk rows with saved output, case {n}")
+        assert_close(rv, dv1[rows], 1e-12, f"dv rows with saved output, case {n}")
+
+    # (e) bf16 bits of a saved output: the bf16 entry points equal the fp64
+    # ones on the widened values, bitwise.
+    rng = np.random.default_rng(160)
+    bits = lambda shape: (rng.standard_normal(shape).astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
+    widen = lambda b: (b.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    q, k, v, do, xo = bits((20, 4, 8)), bits((20, 2, 8)), bits((20, 2, 8)), bits((20, 4, 8)), bits((20, 4, 8))
+    s = rng.standard_normal(4).astype(np.float32)
+    cu = np.array([0, 7, 20], np.int32)
+    wq, wk, wv, wdo, wxo, ws = widen(q), widen(k), widen(v), widen(do), widen(xo), s.astype(np.float64)
+    ga = O.bwd(q, k, v, s, cu, 3, 0.125, do, out_for_D=xo)
+    gb = O.bwd(wq, wk, wv, ws, cu, 3, 0.125, wdo, out_for_D=wxo)
+    assert all(np.array_equal(x, y) for x, y in zip(ga, gb)), "bf16 saved output widening (bwd)"
+    rows = np.array([0, 6, 7, 19])
+    assert np.array_equal(O.bwd_dq_rows(q, k, v, s, cu, 3, 0.125, do, rows, out_for_D=xo),
+                          O.bwd_dq_rows(wq, wk, wv, ws, cu, 3, 0.125, wdo, rows, out_for_D=wxo)), \
+        "bf16 saved output widening (dq rows)"
+    ka = O.bwd_dkv_rows(q, k, v, s, cu, 3, 0.125, do, rows, out_for_D=xo)
+    kb = O.bwd_dkv_rows(wq, wk, wv, ws, cu, 3, 0.125, wdo, rows, out_for_D=wxo)
+    assert np.array_equal(ka[0], kb[0]) and np.array_equal(ka[1], kb[1]), "bf16 saved output widening (dk/dv rows)"
+    assert np.array_equal(O.bwd_dsinks(q, k, v, s, cu, 3, 0.125, do, out_for_D=xo),
+                          O.bwd_dsinks(wq, wk, wv, ws, cu, 3, 0.125, wdo, out_for_D=wxo)), \
+        "bf16 saved output widening (dsinks alone)"
 
 
 ALL_PINS = [
@@ -373,4 +475,5 @@ ALL_PINS = [
     pin_rows_match_full,
     pin_bf16_widening,
     pin_restricted_backward,
+    pin_saved_output_for_D,
 ]

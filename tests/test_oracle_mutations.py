@@ -14,6 +14,9 @@ import pytest
 import oracle
 from tests import oracle_pins
 
+_SAVED_OUT = "const double* o = out_for_D ? out_for_D + (t * Hq + h) * (int64_t)D : orow;"
+
+# name -> (anchor, replacement[, which occurrence of the anchor, default 0])
 MUTATIONS = {
     "sink dropped from the denominator": ("double Z = exp(sink - m);", "double Z = 0.0 * exp(sink - m);"),
     "window one key too wide": ("int64_t lo = t - (int64_t)window + 1;", "int64_t lo = t - (int64_t)window;"),
@@ -29,6 +32,21 @@ MUTATIONS = {
     "dk misses scale": ("dkj[d] += scale * dS * qi[d];", "dkj[d] += dS * qi[d];"),
     "dq uses v": ("dqi[d] += scale * dS * kj[d];", "dqi[d] += scale * dS * vj[d];"),
     "documents not respected": ("int64_t a = cu_seqlens[doc_of(cu_seqlens, B, t)];", "int64_t a = 0;"),
+    # The saved output used for D_i (out_for_D): the same line sits in the
+    # full backward (occurrence 0), the dsinks-only one (1), the dq-rows one
+    # (2) and the dk/dv-rows one (3); each is mutated on its own.
+    **{f"saved output ignored ({where})": (_SAVED_OUT, "const double* o = orow;", n)
+       for n, where in ((0, "bwd"), (1, "dsinks alone"), (2, "dq rows"), (3, "dk/dv rows"))},
+    **{f"saved output indexed [Hq][T] ({where})": (
+        _SAVED_OUT, "const double* o = out_for_D ? out_for_D + ((int64_t)h * T + t) * (int64_t)D : orow;", n)
+       for n, where in ((0, "bwd"), (1, "dsinks alone"), (2, "dq rows"), (3, "dk/dv rows"))},
+    "dsinks alone: sink term sign": ("term[(int64_t)h * T + t] = exp(sinks[h] - lse) * Di;",
+                                     "term[(int64_t)h * T + t] = -exp(sinks[h] - lse) * Di;"),
+    "dsinks alone: lse of the wrong sign": ("term[(int64_t)h * T + t] = exp(sinks[h] - lse) * Di;",
+                                            "term[(int64_t)h * T + t] = exp(sinks[h] + lse) * Di;"),
+    "saved output widened from dout (bf16 bwd)": (
+        "double* od = out_for_D_bf16 ? widen(out_for_D_bf16, (int64_t)T * Hq * D) : NULL;",
+        "double* od = out_for_D_bf16 ? widen(dout, (int64_t)T * Hq * D) : NULL;"),
 }
 
 
@@ -58,10 +76,14 @@ sys.exit(3 if failed else 0)
 
 @pytest.mark.parametrize("name", sorted(MUTATIONS))
 def test_pins_catch_mutation(workdir, name):
-    old, new = MUTATIONS[name]
+    old, new, *nth = MUTATIONS[name]
+    nth = nth[0] if nth else 0
     src = open(oracle.SOURCE).read()
-    assert src.count(old) >= 1, f"mutation anchor not found: {old}"
-    mutated = src.replace(old, new, 1)
+    assert src.count(old) > nth, f"mutation anchor not found: {old} (occurrence {nth})"
+    at = -1
+    for _ in range(nth + 1):
+        at = src.index(old, at + 1)
+    mutated = src[:at] + new + src[at + len(old):]
     tag = "".join(c if c.isalnum() else "_" for c in name)
     path = os.path.join(workdir, f"{tag}.c")
     with open(path, "w") as f:
