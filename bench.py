@@ -312,6 +312,121 @@ def measure_layers(torch, ops, stream, q, k, v, sinks, dout, outs, grads, ws, it
     return res
 
 
+# ------------------------------------------------- long and packed shapes
+EXTRA_WORKLOADS = ("long60k", "varlen64k")
+
+
+def device_inputs(torch, w, seed=11, with_dout=True):
+    """Device-resident N(0,1) bf16 q, k, v (and dout) of a workload's shapes,
+    drawn on the GPU from a seeded generator (the timing does not depend on
+    the exact values, and drawing 0.5 G values on the host would dominate
+    the run), and the workload's own sinks."""
+    g = torch.Generator(device="cuda").manual_seed(seed)
+    mk = lambda *shape: torch.randn(*shape, generator=g, device="cuda").to(torch.bfloat16)  # noqa: E731
+    t = {"q": mk(w.T, w.Hq, w.D), "k": mk(w.T, w.Hkv, w.D), "v": mk(w.T, w.Hkv, w.D),
+         "sinks": torch.from_numpy(w.sinks_only()).cuda()}
+    if with_dout:
+        t["dout"] = mk(w.T, w.Hq, w.D)
+    t["cu"] = None if w.uniform_seqlen is not None else torch.from_numpy(w.cu_seqlens).cuda()
+    return t
+
+
+def layer_calls(ops, w, t, stream, window, bufs):
+    """(forward call, backward call) of one layer of workload w on the
+    device tensors t, writing into bufs = (out, lse, dq, dk, dv, dsinks, ws)."""
+    o, l, dq, dk, dv, ds, ws = bufs
+    if w.uniform_seqlen is not None:
+        kw = dict(batch=w.batch, max_seqlen=w.uniform_seqlen, stream=stream)
+    else:
+        kw = dict(max_seqlen=w.max_seqlen, stream=stream)
+    f = lambda: ops.fwd(t["q"], t["k"], t["v"], t["sinks"], t["cu"], window, w.scale, out=o, lse=l, **kw)  # noqa
+    b = lambda: ops.bwd(t["q"], t["k"], t["v"], t["sinks"], o, l, t["dout"], t["cu"], window, w.scale, dq=dq,  # noqa
+                        dk=dk, dv=dv, dsinks=ds, workspace=ws, **kw)
+    return f, b
+
+
+def layer_buffers(torch, ops, w, t):
+    q, k = t["q"], t["k"]
+    ws = torch.empty((ops.bwd_workspace_size(w.T, w.Hq, w.Hkv, w.D, w.batch, w.max_seqlen),), dtype=torch.uint8,
+                     device="cuda")
+    return (torch.empty_like(q), torch.empty((w.Hq, w.T), dtype=torch.float32, device="cuda"), torch.empty_like(q),
+            torch.empty_like(k), torch.empty_like(k), torch.empty((w.Hq,), dtype=torch.float32, device="cuda"), ws)
+
+
+def measure_extra(torch, ops, stream, iters=5):
+    """Forward and backward of the long-context (one 61,440-token document,
+    sinks ~N(0, 2^2)) and packed-document (65,536 tokens in documents of
+    ~U[256, 8192] tokens) workloads, window 128 and full causal, each call
+    timed alone with CUDA events on the launching stream (mean of `iters`
+    after 2 warm-up calls; every input exceeds the L2, so no flush).  Full
+    causal: TFLOP/s on the counted pairs and % of the measured bf16 peak;
+    window 128: GB/s of the layer's minimum bytes against the HBM peak."""
+    peak, hbm, kind = read_peaks()
+    nb = lambda *ts: sum(x.numel() * x.element_size() for x in ts if x is not None)  # noqa: E731
+    res = {}
+    for base in EXTRA_WORKLOADS:
+        w = synth.workload(f"{base}:full")
+        t = device_inputs(torch, w)
+        bufs = layer_buffers(torch, ops, w, t)
+        o, l, dq, dk, dv, ds, _ = bufs
+        entry = {"workload": f"{base}: T={w.T} in {w.batch} document(s) (max {w.max_seqlen}), Hq=64 Hkv=8 D=64, "
+                             f"sinks ~N(0, {w.sink_std:g}^2); inputs drawn on the GPU",
+                 "layers": []}
+        for window in (128, 0):
+            f, b = layer_calls(ops, w, t, stream, window, bufs)
+            p = pairs(w.cu_seqlens, window, w.Hq)
+            lay = {"window": window}
+            for name, fn, flops, mb in (
+                    ("fwd", f, 4 * D * p, nb(t["q"], t["k"], t["v"], t["sinks"], o, l)),
+                    ("bwd", b, 10 * D * p, nb(t["q"], t["k"], t["v"], t["sinks"], o, l, t["dout"], dq, dk, dv, ds))):
+                for _ in range(2):
+                    fn()
+                torch.cuda.synchronize()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                for _ in range(iters):
+                    fn()
+                e1.record(stream)
+                torch.cuda.synchronize()
+                ms = e0.elapsed_time(e1) / iters
+                lay[name] = {"ms": ms, "tflops": flops / ms / 1e9, "pct_of_peak": 100.0 * flops / ms / 1e9 / peak,
+                             "min_bytes": mb, "GBps": mb / ms / 1e6, "hbm_frac": mb / ms / 1e6 / hbm}
+            entry["layers"].append(lay)
+        entry["peak_TFLOPs"], entry["peak_GBps"], entry["peak_source"] = peak, hbm, f"{kind} bf16_tflops / hbm_gbs"
+        res[base] = entry
+        del t, bufs
+        torch.cuda.empty_cache()
+    if ops.device_error() != 0:
+        raise RuntimeError("a kernel reported a timed-out wait")
+    return res
+
+
+def run_profile_case(args):
+    """--profile-case KIND:WORKLOAD:LAYER (e.g. fwd:long60k:full,
+    bwd:prefill4k:w128): two calls of one entry point on one workload, for an
+    ncu capture of its kernels (capture the second: -s <launches of one
+    call>).  Prints nothing but a done line."""
+    import torch
+    from sink_sliding_window_b200 import build, ops
+    kind, name = args.profile_case.split(":", 1)
+    torch.cuda.set_device(0)
+    build.build()
+    ops.load()
+    w = synth.workload(name)
+    t = device_inputs(torch, w, with_dout=kind == "bwd")
+    stream = torch.cuda.current_stream()
+    bufs = layer_buffers(torch, ops, w, t)
+    f, b = layer_calls(ops, w, t, stream, w.window, bufs)
+    if kind == "bwd":
+        f()
+    for _ in range(2):
+        (f if kind == "fwd" else b)()
+    torch.cuda.synchronize()
+    if ops.device_error() != 0:
+        raise RuntimeError("a kernel reported a timed-out wait")
+    print(f"profile case {args.profile_case} done", flush=True)
+
+
 # ----------------------------------------------------------- aggregation
 def max_over_ranks(x, dist, device):
     """Largest value of x over all ranks (the slowest rank's time); x itself
@@ -502,6 +617,7 @@ def run_ours(args, rank, world, torch, dist):
 
     layers = measure_layers(torch, ops, stream, q, k, v, sinks, dout, outs, grads, ws)
     decode = measure_decode(torch, ops, stream) if not args.skip_decode else None
+    extra = measure_extra(torch, ops, stream) if not args.skip_extra else None
 
     if rank != 0:
         return
@@ -526,6 +642,8 @@ def run_ours(args, rank, world, torch, dist):
     line["layers"] = layers
     if decode is not None:
         line["decode"] = decode
+    if extra is not None:
+        line.update(extra)
     if world == 1 and not args.skip_cpu_baseline:
         secs, cflops, desc, threads = oracle_sample(S, 2048)
         line["cpu_baseline"] = {"value": cflops / secs / 1e12, "unit": "TFLOP/s", "cores": threads,
@@ -542,6 +660,10 @@ def main(argv=None):
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--skip-cpu-baseline", action="store_true")
     ap.add_argument("--skip-decode", action="store_true", help="do not time sink_attn_decode after the step")
+    ap.add_argument("--skip-extra", action="store_true",
+                    help="do not time the long-context and packed-document layers after the step")
+    ap.add_argument("--profile-case", default=None,
+                    help="KIND:WORKLOAD:LAYER, e.g. fwd:long60k:full: only run two calls of one entry point (for ncu)")
     ap.add_argument("--budget-s", type=float, default=120.0,
                     help="--impl reference: seconds all warmup + timed oracle steps should take")
     args = ap.parse_args(argv)
@@ -552,6 +674,9 @@ def main(argv=None):
     rank = int(os.environ.get("RANK", "0"))
     if args.impl == "reference":
         run_reference(args, rank)
+        return 0
+    if args.profile_case:
+        run_profile_case(args)
         return 0
     import torch
 

@@ -94,11 +94,16 @@ class Workload:
             a["q"] = normal_bf16(self.seed, "q", (self.T, self.Hq, self.D))
             a["k"] = normal_bf16(self.seed, "k", (self.T, self.Hkv, self.D))
             a["v"] = normal_bf16(self.seed, "v", (self.T, self.Hkv, self.D))
-            s = _rng(self.seed, "sinks").standard_normal(size=(self.Hq,), dtype=np.float32)
-            a["sinks"] = (s * np.float32(self.sink_std)).astype(np.float32)
+            a["sinks"] = self.sinks_only()
         if with_dout and "dout" not in a:
             a["dout"] = normal_bf16(self.seed, "dout", (self.T, self.Hq, self.D))
         return a
+
+    def sinks_only(self) -> np.ndarray:
+        """The workload's sinks (the same draw generate() makes), without
+        generating q, k, v."""
+        s = _rng(self.seed, "sinks").standard_normal(size=(self.Hq,), dtype=np.float32)
+        return (s * np.float32(self.sink_std)).astype(np.float32)
 
     def sample_rows(self, n: int) -> np.ndarray:
         """Seeded sample of query tokens: for each of the first 8 documents
