@@ -264,7 +264,7 @@ def measure_decode(torch, ops, stream, iters=20):
         kv = Bd * keys * HKV * D * 2 * (1 if f8 else 2)  # K and V bytes as stored
         res.append({"workload": name, "us": ms * 1e3, "kv_bytes": kv, "achieved_GBps": kv / ms / 1e6,
                     "peak_GBps": hbm, "frac": kv / ms / 1e6 / hbm, "peak_source": f"{kind} hbm_gbs",
-                    "launches": ops.decode_launches(Bd, Lq, C, L0 + Lq, HQ, HKV)})
+                    "launches": ops.decode_launches(Bd, Lq, C, L0 + Lq, HQ, HKV, W)})
     return res
 
 

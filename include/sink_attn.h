@@ -200,8 +200,8 @@ size_t sink_attn_decode_workspace_size(const sink_attn_decode_dims* dims, int wi
  * Supported: D = 64, G = Hq / Hkv a power of two with G * new_tokens <= 64.
  * `workspace`: caller-owned device memory of at least
  * sink_attn_decode_workspace_size(dims, window) bytes, 256-byte aligned.
- * batch = 0 is a no-op.  Launches three kernels (append, attend, combine)
- * on `stream`. */
+ * batch = 0 is a no-op.  Launches two or three kernels on `stream` (see
+ * sink_attn_decode_launches). */
 sink_attn_status sink_attn_decode(const sink_attn_decode_dims* dims,
                                   const void* q, const void* k_new, const void* v_new,
                                   void* k_cache, void* v_cache, const int* cache_seqlens,
@@ -234,8 +234,11 @@ sink_attn_status sink_attn_decode_e4m3(const sink_attn_decode_dims* dims,
                                        void* workspace, size_t workspace_bytes,
                                        void* stream);
 
-/* Number of kernels one sink_attn_decode call launches (0 when batch = 0). */
-int sink_attn_decode_launches(const sink_attn_decode_dims* dims);
+/* Number of kernels one sink_attn_decode / sink_attn_decode_e4m3 call
+ * launches for these sizes and window (0 when batch = 0): append, attend and
+ * combine, or only the first two when one CTA per (sequence, key/value head)
+ * covers the cache (the attend kernel then finishes the rows itself). */
+int sink_attn_decode_launches(const sink_attn_decode_dims* dims, int window);
 
 /* Human-readable name of a status code (static string, never NULL). */
 const char* sink_attn_status_string(sink_attn_status s);

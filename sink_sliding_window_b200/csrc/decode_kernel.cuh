@@ -29,7 +29,9 @@
 // Softmax is invariant to the order of the keys, so slots are visited in
 // slot order; each key's position (and so its mask) follows from the slot.
 // Each split writes (O, l, m) partials; the combine kernel merges them and
-// adds the sink's e^{s-m} once.
+// adds the sink's e^{s-m} once.  With a single split (the cache of every
+// (sequence, key/value head) fits one CTA's share of the grid) the attention
+// kernel finishes the rows itself and the combine launch is skipped.
 //
 // e4m3 cache variant (kF8): the cache holds FP8 e4m3 codes with one
 // dequantisation scale per key/value head (k = code * k_scale[g], likewise
@@ -80,6 +82,8 @@ struct DecParams {
   float* o_part;                    // [batch][Hkv][n_split][64 rows][64] unnormalised O
   float* m_part;                    // [batch][Hkv][n_split][64 rows] reference max (log2 units)
   float* l_part;                    // [batch][Hkv][n_split][64 rows] sum of P
+  __nv_bfloat16* out;               // n_split == 1: the attention kernel writes out and lse itself
+  float* lse_out;
 };
 
 struct DecCtl {
@@ -650,7 +654,55 @@ __global__ void __launch_bounds__(kF8 ? kDecThreads8 : kDecThreads, (kF8 && kR >
     if (have) have = mbar_wait(&ctl->o_full, 0, abort, &g_device_error, kDevErrTimeoutEpilogue);
     have = __all_sync(0xffffffffu, have);
     if (have) tc_fence_after();
-    if (warp < 3) {
+    if (p.n_split == 1) {
+      // One split covers the whole cache: finish here (what the combine
+      // kernel does for several splits), m = max(s, m_0),
+      // l = e^{s-m} + l_0 e^{m_0-m}, out = O_0 e^{m_0-m} / l, lse = m + ln l
+      // (exponents in base 2), and skip the combine launch.
+      if (warp < 3) {
+        uint32_t o[kR];
+        if (have) {
+          __syncwarp();
+          dec_tmem_ld<kR>(tmem + lane_base + kDecTmemO, o);
+        }
+        if (kl == 64) {
+          // Lane 64: the row sums -> per-row output factor and lse.
+#pragma unroll
+          for (int n = 0; n < kR; ++n) {
+            if (n >= p.R) continue;
+            const int h = (w.g << p.G_log2) + (n & (p.G - 1));
+            const float s2 = __ldg(p.sinks + h) * kLog2e;
+            const float m0 = (have && w.n > 0) ? ctl->m_ref[n] : -INFINITY;
+            const float m = fmaxf(s2, m0);
+            float l = 0.f, f = 0.f;
+            if (m != -INFINITY) {
+              if (s2 != -INFINITY) l = ex2_approx(s2 - m);
+              if (m0 != -INFINITY) {
+                f = ex2_approx(m0 - m);
+                l = fmaf(__uint_as_float(o[n]), f, l);
+              }
+            }
+            ctl->alpha[n] = l > 0.f ? f / l : 0.f;
+            const int t = n >> p.G_log2;
+            p.lse_out[static_cast<size_t>(h) * (p.batch * p.Lq) + w.b * p.Lq + t] =
+                l > 0.f ? (m + __log2f(l)) * kLn2 : -INFINITY;
+          }
+        }
+        named_barrier(2, 96);  // warps 0-2: the factors are in shared memory
+        if (warp < 2) {
+          // Lanes 0..63: head dim kl of every query row.
+          const float vs = kF8 ? __ldg(p.v_scale + w.g) : 1.f;
+#pragma unroll
+          for (int n = 0; n < kR; ++n) {
+            if (n >= p.R) continue;
+            const int h = (w.g << p.G_log2) + (n & (p.G - 1));
+            const int t = n >> p.G_log2;
+            const float y = have ? __uint_as_float(o[n]) * vs * ctl->alpha[n] : 0.f;
+            p.out[(static_cast<size_t>(w.b * p.Lq + t) * p.Hq + h) * kHeadDim + kl] = __float2bfloat16_rn(y);
+          }
+        }
+      }
+    } else if (warp < 3) {
       uint32_t o[kR];
       if (have) {
         __syncwarp();
@@ -670,7 +722,7 @@ __global__ void __launch_bounds__(kF8 ? kDecThreads8 : kDecThreads, (kF8 && kR >
           if (n < p.R) p.l_part[cta * kDecRows + n] = have ? __uint_as_float(o[n]) : 0.f;
       }
     }
-    if (kl < p.R) p.m_part[cta * kDecRows + kl] = (w.n > 0) ? ctl->m_ref[kl] : -INFINITY;
+    if (p.n_split > 1 && kl < p.R) p.m_part[cta * kDecRows + kl] = (w.n > 0) ? ctl->m_ref[kl] : -INFINITY;
   }
 
   tc_fence_before();

@@ -112,6 +112,8 @@ sink_attn_status plan_decode(const sink_attn_decode_dims* d, int window, float s
   p.sinks = nullptr;
   p.k_scale = p.v_scale = nullptr;
   p.o_part = p.m_part = p.l_part = nullptr;
+  p.out = nullptr;
+  p.lse_out = nullptr;
   // Upper bound on the 128-slot tiles one sequence scans.
   int64_t slots = std::min<int64_t>(d->cache_capacity, d->max_seqlen);
   if (p.window > 0) slots = std::min<int64_t>(slots, static_cast<int64_t>(p.window) + d->new_tokens - 1 + kDecTile);
@@ -355,10 +357,10 @@ size_t sink_attn_decode_workspace_size(const sink_attn_decode_dims* d, int windo
   return plan.total;
 }
 
-int sink_attn_decode_launches(const sink_attn_decode_dims* d) {
+int sink_attn_decode_launches(const sink_attn_decode_dims* d, int window) {
   DecPlan plan;
-  if (plan_decode(d, 0, 1.f, &plan) != SINK_ATTN_OK) return 0;
-  return d->batch > 0 ? 3 : 0;
+  if (plan_decode(d, window, 1.f, &plan) != SINK_ATTN_OK) return 0;
+  return d->batch > 0 ? (plan.p.n_split > 1 ? 3 : 2) : 0;
 }
 
 }  // extern "C"
@@ -392,6 +394,8 @@ sink_attn_status decode_impl(const sink_attn_decode_dims* d, const void* q, cons
   p.o_part = reinterpret_cast<float*>(ws + plan.o_off);
   p.m_part = reinterpret_cast<float*>(ws + plan.m_off);
   p.l_part = reinterpret_cast<float*>(ws + plan.l_off);
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.lse_out = lse;
 
   CUtensorMap tq, tk, tv;
   if (!make_map_3d(&tq, q, kHeadDim, p.Hq, p.batch * p.Lq, p.G, p.Lq)) return SINK_ATTN_ERR_CUDA;
@@ -431,9 +435,11 @@ sink_attn_status decode_impl(const sink_attn_decode_dims* d, const void* q, cons
         static_cast<uint4*>(v_cache));
   }
   kern<<<static_cast<unsigned>(ctas), e4m3 ? kDecThreads8 : kDecThreads, smem, st_>>>(tq, tk, tv, p);
-  const long long rows = static_cast<long long>(p.batch) * p.Lq * p.Hq;
-  sink_attn_decode_combine_kernel<<<static_cast<unsigned>((rows + 3) / 4), 128, 0, st_>>>(
-      p, static_cast<__nv_bfloat16*>(out), lse);
+  if (p.n_split > 1) {
+    const long long rows = static_cast<long long>(p.batch) * p.Lq * p.Hq;
+    sink_attn_decode_combine_kernel<<<static_cast<unsigned>((rows + 3) / 4), 128, 0, st_>>>(
+        p, static_cast<__nv_bfloat16*>(out), lse);
+  }
   return cudaPeekAtLastError() == cudaSuccess ? SINK_ATTN_OK : SINK_ATTN_ERR_CUDA;
 }
 

@@ -89,7 +89,7 @@ def load():
         L.sink_attn_decode_e4m3.restype = I
         L.sink_attn_decode_workspace_size.argtypes = [DD, I]
         L.sink_attn_decode_workspace_size.restype = ctypes.c_size_t
-        L.sink_attn_decode_launches.argtypes = [DD]
+        L.sink_attn_decode_launches.argtypes = [DD, I]
         L.sink_attn_decode_launches.restype = I
         L.sink_attn_selftest_wait.argtypes = [ctypes.c_ulonglong, P, P]
         L.sink_attn_selftest_wait.restype = I
@@ -194,9 +194,9 @@ def decode_workspace_size(batch, new_tokens, cache_capacity, max_seqlen, Hq, Hkv
     return int(load().sink_attn_decode_workspace_size(ctypes.byref(d), int(window)))
 
 
-def decode_launches(batch, new_tokens, cache_capacity, max_seqlen, Hq, Hkv, D=64) -> int:
+def decode_launches(batch, new_tokens, cache_capacity, max_seqlen, Hq, Hkv, window=0, D=64) -> int:
     d = decode_dims(batch, new_tokens, cache_capacity, max_seqlen, Hq, Hkv, D)
-    return int(load().sink_attn_decode_launches(ctypes.byref(d)))
+    return int(load().sink_attn_decode_launches(ctypes.byref(d), int(window)))
 
 
 def decode(q, k_new, v_new, k_cache, v_cache, cache_seqlens, sinks, window=0, scale=None, *, max_seqlen=None,

@@ -154,6 +154,13 @@ def test_decode_empty_batch_is_noop(L):
     assert call_decode(L, ddims(B=0), [None] * 7, ws=None, ws_bytes=0) == 0
     assert ops.decode_launches(0, 1, 256, 257, 64, 8) == 0
     assert ops.decode_launches(4, 1, 256, 257, 64, 8) == 3
+    # One CTA per (sequence, key/value head) covers the cache (64 x 8 CTAs
+    # already fill the grid; the split plan keeps one): the attention kernel
+    # finishes the rows and the combine launch is skipped.
+    assert ops.decode_launches(64, 1, 256, 257, 64, 8) == 2
+    assert ops.decode_launches(64, 1, 128, 8192, 64, 8, window=128) == 2
+    # A long cache is split over several CTAs and combined.
+    assert ops.decode_launches(64, 1, 8192, 8192, 64, 8) == 3
 
 
 def test_binding_refuses_host_tensors():

@@ -150,6 +150,7 @@ def test_gpt_oss_decode_full_size(ops, window, C):
 def test_launch_count(ops):
     assert ops.decode_launches(4, 1, 256, 257, 64, 8) == 3
     assert ops.decode_launches(0, 1, 256, 257, 64, 8) == 0
+    assert ops.decode_launches(64, 1, 128, 8192, 64, 8, window=128) == 2
 
 
 # ----------------------------------------------------------------- e4m3 cache
@@ -242,5 +243,10 @@ def test_e4m3_cache_heavy_tailed(ops, window):
     _run_e4m3(ops, [1000, 2000, 4095, 3], 1, 16, 2, 4096, window, seed=90 + window, heavy=True)
 
 
-def test_e4m3_cache_gpt_oss_full_size(ops):
-    _run_e4m3(ops, [8191] * 62 + [0, 4000], 1, 64, 8, 8192, 0, seed=80, seqs=[0, 31, 62, 63])
+@pytest.mark.parametrize("window,C", [(0, 8192), (128, 128)])
+def test_e4m3_cache_gpt_oss_full_size(ops, window, C):
+    """gpt-oss heads, 64 sequences: the full-causal layer's 8192-slot cache
+    is split over several CTAs and combined; the window-128 layer's 128-slot
+    ring fits one CTA per (sequence, key/value head), which then finishes
+    the rows itself (no combine launch)."""
+    _run_e4m3(ops, [8191] * 62 + [0, 4000], 1, 64, 8, C, window, seed=80, seqs=[0, 31, 62, 63])
