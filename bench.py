@@ -203,6 +203,8 @@ DECODE_CASES = (
     ("decode 64 seqs x 8191 cached + 1 new, window-128 layer, 128-slot ring", 64, 8191, 1, 128, 128, False),
     ("decode 64 seqs x 8191 cached + 1 new, full-causal layer, linear 8192-slot e4m3 cache", 64, 8191, 1, 8192, 0,
      True),
+    ("decode 64 seqs x 8191 cached + 1 new, full-causal layer, linear 8192-slot e4m3 cache, FP8 PV product", 64, 8191,
+     1, 8192, 0, "f8pv"),
 )
 
 
@@ -241,7 +243,7 @@ def measure_decode(torch, ops, stream, iters=20):
         def call():
             if f8:
                 ops.decode_e4m3(q, kn, vn, kc, vc, sl, k_scale, v_scale, sinks, W, 0.125, max_seqlen=L0 + Lq, out=out,
-                                lse=lse, workspace=ws, stream=stream)
+                                lse=lse, workspace=ws, stream=stream, f8pv=f8 == "f8pv")
             else:
                 ops.decode(q, kn, vn, kc, vc, sl, sinks, W, 0.125, max_seqlen=L0 + Lq, out=out, lse=lse,
                            workspace=ws, stream=stream)

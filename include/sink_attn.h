@@ -234,6 +234,31 @@ sink_attn_status sink_attn_decode_e4m3(const sink_attn_decode_dims* dims,
                                        void* workspace, size_t workspace_bytes,
                                        void* stream);
 
+/* Decode over an FP8 (e4m3) cache with the PV product on the FP8 tensor-core
+ * path (tcgen05 kind::f8f6f4).  Arguments, cache layout, quantisation of the
+ * new tokens and workspace as for sink_attn_decode_e4m3().  The value codes
+ * are read as stored (not widened to fp16), and the unnormalised weights
+ * p_j = 2^(x_j - m) of each row (m the kernel's running reference of the
+ * row, p_j <= 2^8) are rounded to e4m3 (nearest even, saturating) before
+ * the MMA; the row sums use the same rounded weights, so every output row is
+ * still a convex combination of its cached values.  The rounding moves each
+ * weight by at most 2^-4 of itself (e4m3's 3 mantissa bits; below e4m3's
+ * normal range, 2^-6, by at most 2^-10), which bounds the extra error of a
+ * row with normalised weights pi_j by
+ *   |out - exact| <= 2^-4 sum_j pi_j |v_j - out| + 2^-10 max_j pi_j sum_j |v_j - out|
+ *   |lse - exact| <= 2^-4 + 2^-10 max_j pi_j * (keys seen)
+ * on top of sink_attn_decode_e4m3's own rounding.  The logits keep the fp16
+ * path of sink_attn_decode_e4m3 (keys widened to fp16, queries converted to
+ * fp16): e4m3 queries would move every logit by up to 2^-4 of its terms. */
+sink_attn_status sink_attn_decode_e4m3_f8pv(const sink_attn_decode_dims* dims,
+                                            const void* q, const void* k_new, const void* v_new,
+                                            void* k_cache, void* v_cache, const int* cache_seqlens,
+                                            const float* k_scale, const float* v_scale,
+                                            const float* sinks, int window, float scale,
+                                            void* out, float* lse,
+                                            void* workspace, size_t workspace_bytes,
+                                            void* stream);
+
 /* Number of kernels one sink_attn_decode / sink_attn_decode_e4m3 call
  * launches for these sizes and window (0 when batch = 0): append, attend and
  * combine, or only the first two when one CTA per (sequence, key/value head)

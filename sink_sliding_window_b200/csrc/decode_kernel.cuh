@@ -113,6 +113,11 @@ constexpr size_t kDecSmemBytes = 1024 /*alignment slack*/ + kDecQBytes + 2 * kDe
                                  kDecKvBytes /*ones*/ + kDecPBytes + sizeof(DecCtl);
 constexpr size_t kDecSmemBytes8 = 1024 + kDecQBytes + 2 * kDecStages8 * kDecKv8Bytes + 2 * kDecKvBytes /*fp16 V x2*/ +
                                   kDecKvBytes /*ones*/ + kDecPBytes + sizeof(DecCtl);
+// e4m3 cache with the PV product in FP8: no widened V tiles; the ones tile
+// and P^T are e4m3 bytes, [128 slots][64].
+constexpr int kDecP8Bytes = kDecTile * kDecRows;
+constexpr size_t kDecSmemBytesPv8 =
+    1024 + kDecQBytes + 2 * kDecStages8 * kDecKv8Bytes + kDecKv8Bytes /*ones*/ + kDecP8Bytes + sizeof(DecCtl);
 
 // Slot range of one CTA: [z0, z0 + 128 n) in 128-slot tiles.
 struct DecWork {
@@ -255,6 +260,33 @@ __device__ __forceinline__ void dec_issue_pv(uint32_t tmem_o, uint32_t v_addr, u
   }
 }
 
+// O^T (+)= [V | 1]^T P^T in FP8 (tcgen05 kind::f8f6f4, e4m3 A and B, fp32
+// accumulate, K = 32 slots per MMA): A (M = 128) read MN-major straight from
+// the e4m3 V byte tile (M rows 0..63: 64 bytes per slot, 64-byte swizzle) and
+// the e4m3 ones tile (M rows 64..127, through the leading-byte offset); B =
+// the first kN query rows of P^T, e4m3 bytes [slots][64 rows], MN-major,
+// 64-byte swizzle.
+template <int kN>
+__device__ __forceinline__ void dec_issue_pv_f8(uint32_t tmem_o, uint32_t v_addr, uint32_t ones_addr,
+                                                uint32_t p_addr, bool accumulate) {
+  constexpr uint32_t idesc = make_idesc_e4m3(kDecTile, kN, 1, 1);
+  const uint32_t lbo = ones_addr - v_addr;
+#pragma unroll
+  for (int kk = 0; kk < kDecTile / 32; ++kk) {
+    const uint64_t a = make_sdesc_sw64(v_addr + kk * 2048, lbo, 512);
+    const uint64_t b = make_sdesc_sw64(p_addr + kk * 2048, kDecP8Bytes, 512);
+    mma_ss_f8(tmem_o, a, b, idesc, (accumulate || kk > 0) ? 1u : 0u);
+  }
+}
+
+// Two fp32 -> two e4m3 codes (low byte first), rounded to nearest even and
+// saturated to +-448.
+__device__ __forceinline__ uint32_t dec_f32x2_to_e4m3x2(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
 // The 128 softmax threads (warps 0-3) on hardware barrier 1: an OR of one
 // predicate over them, and a plain barrier.  Every softmax thread executes the
 // same sequence of these (see the softmax loop), so none is left waiting.
@@ -293,11 +325,14 @@ __device__ __forceinline__ void dec_tmem_st(uint32_t taddr, const uint32_t* r) {
 }
 
 // kR: query rows handled in registers (8, 16, 32 or 64; >= G * Lq).
-// kF8: the cache holds e4m3 codes (see the file comment).
-template <int kR, bool kF8>
-__global__ void __launch_bounds__(kF8 ? kDecThreads8 : kDecThreads, (kF8 && kR > 16) ? 1 : 2)
+// kMode: 0 bf16 cache; 1 e4m3 cache (see the file comment); 2 e4m3 cache
+// with the PV product in FP8 (P rounded to e4m3; V read as stored).
+template <int kR, int kMode>
+__global__ void __launch_bounds__(kMode ? kDecThreads8 : kDecThreads, (kMode && kR > 16) ? 1 : 2)
     sink_attn_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                             const __grid_constant__ CUtensorMap tm_v, const DecParams p) {
+  constexpr bool kF8 = kMode >= 1;
+  constexpr bool kPv8 = kMode == 2;
   constexpr int kStages = kF8 ? kDecStages8 : kDecStages;
   constexpr int kTileB = kF8 ? kDecKv8Bytes : kDecKvBytes;  // bytes of one staged K or V tile
   constexpr int kThreads = kF8 ? kDecThreads8 : kDecThreads;
@@ -307,9 +342,9 @@ __global__ void __launch_bounds__(kF8 ? kDecThreads8 : kDecThreads, (kF8 && kR >
   uint8_t* sK = smem;                                   // stages of K tiles
   uint8_t* sV = sK + kStages * kTileB;                  // stages of V tiles
   uint8_t* sVb = sV + kStages * kTileB;                 // e4m3 cache: two widened V tiles (fp16)
-  uint8_t* sOnes = sVb + (kF8 ? 2 * kDecKvBytes : 0);   // [128][64] ones
-  uint8_t* sP = sOnes + kDecKvBytes;                    // P^T
-  uint8_t* sQ = sP + kDecPBytes;                        // Q rows (8 KB, 1024-aligned)
+  uint8_t* sOnes = sVb + ((kF8 && !kPv8) ? 2 * kDecKvBytes : 0);  // [128][64] ones
+  uint8_t* sP = sOnes + (kPv8 ? kDecKv8Bytes : kDecKvBytes);      // P^T
+  uint8_t* sQ = sP + (kPv8 ? kDecP8Bytes : kDecPBytes);           // Q rows (8 KB, 1024-aligned)
   DecCtl* ctl = reinterpret_cast<DecCtl*>(sQ + kDecQBytes);
   volatile int* abort = &ctl->abort;
   const int warp = threadIdx.x >> 5;
@@ -324,7 +359,7 @@ __global__ void __launch_bounds__(kF8 ? kDecThreads8 : kDecThreads, (kF8 && kR >
       mbar_init(&ctl->k_full[s], 1);
       mbar_init(&ctl->k_empty[s], kF8 ? kDecTile : 1);  // e4m3: freed by the 128 widening threads
       mbar_init(&ctl->v_full[s], 1);
-      mbar_init(&ctl->v_empty[s], kF8 ? kDecTile : 1);
+      mbar_init(&ctl->v_empty[s], (kF8 && !kPv8) ? kDecTile : 1);  // FP8 PV: released by the MMA
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&ctl->s_full[b], 1);
@@ -348,13 +383,14 @@ __global__ void __launch_bounds__(kF8 ? kDecThreads8 : kDecThreads, (kF8 && kR >
   // Constant operands written by the threads: the ones tile, zeroed P^T and
   // zeroed Q padding rows (the TMA fills rows [0, R)).
   {
-    const uint32_t one2 = kF8 ? 0x3C003C00u : 0x3F803F80u;  // 1.0 in fp16 / bf16 pairs
+    // 1.0 in e4m3 codes / fp16 pairs / bf16 pairs
+    const uint32_t one2 = kPv8 ? 0x38383838u : (kF8 ? 0x3C003C00u : 0x3F803F80u);
     const uint4 ones = make_uint4(one2, one2, one2, one2);
     const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
-    for (int i = threadIdx.x; i < kDecKvBytes / 16; i += kThreads) {
-      reinterpret_cast<uint4*>(sOnes)[i] = ones;
-      reinterpret_cast<uint4*>(sP)[i] = zero;
-    }
+    constexpr int kOnesChunks = (kPv8 ? kDecKv8Bytes : kDecKvBytes) / 16;
+    constexpr int kPChunks = (kPv8 ? kDecP8Bytes : kDecPBytes) / 16;
+    for (int i = threadIdx.x; i < kOnesChunks; i += kThreads) reinterpret_cast<uint4*>(sOnes)[i] = ones;
+    for (int i = threadIdx.x; i < kPChunks; i += kThreads) reinterpret_cast<uint4*>(sP)[i] = zero;
     for (int i = p.R * 8 + threadIdx.x; i < kDecQBytes / 16; i += kThreads) reinterpret_cast<uint4*>(sQ)[i] = zero;
     fence_proxy_async_smem();
   }
@@ -423,16 +459,23 @@ __global__ void __launch_bounds__(kF8 ? kDecThreads8 : kDecThreads, (kF8 && kR >
         if (i >= 1) {
           const int j = i - 1;
           const int s = j % kStages;
-          // e4m3: V_j widened into fp16 tile j % 2 (v_ready).
+          // e4m3: V_j widened into fp16 tile j % 2 (v_ready); FP8 PV: the
+          // V bytes as loaded (the softmax threads zero empty slots' rows
+          // before their P^T arrival).
           ok = mbar_wait(&ctl->p_full, j & 1, abort, &g_device_error, kDevErrTimeoutMma) &&
-               (kF8 ? mbar_wait(&ctl->v_ready[j & 1], (j >> 1) & 1, abort, &g_device_error, kDevErrTimeoutMma)
+               ((kF8 && !kPv8)
+                    ? mbar_wait(&ctl->v_ready[j & 1], (j >> 1) & 1, abort, &g_device_error, kDevErrTimeoutMma)
                     : mbar_wait(&ctl->v_full[s], (j / kStages) & 1, abort, &g_device_error, kDevErrTimeoutMma));
           if (!ok) break;
           tc_fence_after();
-          dec_issue_pv<kF8, kN>(tO, kF8 ? smem_u32(sVb + (j & 1) * kDecKvBytes) : smem_u32(sV + s * kDecKvBytes),
-                            ones_addr, p_addr, j > 0);
+          if constexpr (kPv8) {
+            dec_issue_pv_f8<kN>(tO, smem_u32(sV + s * kTileB), ones_addr, p_addr, j > 0);
+          } else {
+            dec_issue_pv<kF8, kN>(tO, kF8 ? smem_u32(sVb + (j & 1) * kDecKvBytes) : smem_u32(sV + s * kDecKvBytes),
+                                  ones_addr, p_addr, j > 0);
+          }
           tc_commit(&ctl->pv_done[j & 1]);
-          if constexpr (!kF8) tc_commit(&ctl->v_empty[s]);
+          if constexpr (!kF8 || kPv8) tc_commit(&ctl->v_empty[s]);
         }
       }
       if (ok) tc_commit(&ctl->o_full);
@@ -478,6 +521,7 @@ __global__ void __launch_bounds__(kF8 ? kDecThreads8 : kDecThreads, (kF8 && kR >
         mbar_arrive(&ctl->k_empty[s]);
         tc_fence_before();
         mbar_arrive(&ctl->kt_full[b]);
+        if constexpr (kPv8) continue;  // the FP8 PV reads the V bytes as loaded
         // V_i -> fp16 tile i % 2, whose last reader was the PV MMA of tile
         // i-2.  A slot that holds no token may hold any bits (NaN included)
         // and its V row is still multiplied by P = 0: it becomes zeros.
@@ -595,14 +639,20 @@ __global__ void __launch_bounds__(kF8 ? kDecThreads8 : kDecThreads, (kF8 && kR >
         }
       }
       if (!ok) continue;
-      // P^T row of this key, packed to bf16 pairs (rows 2c, 2c+1).
+      // P^T row of this key, packed to bf16 / fp16 pairs (rows 2c, 2c+1),
+      // or (FP8 PV) to e4m3 codes, four rows per word (rows 4c..4c+3).
       uint32_t pk[kR / 2];
 #pragma unroll
       for (int c = 0; c < kR / 2; ++c) {
         const float m0 = mref(2 * c), m1 = mref(2 * c + 1);
         const float e0 = ex2_approx(x[2 * c] - (m0 == -INFINITY ? 0.f : m0));
         const float e1 = ex2_approx(x[2 * c + 1] - (m1 == -INFINITY ? 0.f : m1));
-        pk[c] = kF8 ? pack_f16x2(e0, e1) : pack_bf16x2(e0, e1);
+        if constexpr (kPv8) {
+          const uint32_t codes = dec_f32x2_to_e4m3x2(e0, e1);
+          pk[c / 2] = (c & 1) ? (pk[c / 2] | (codes << 16)) : codes;
+        } else {
+          pk[c] = kF8 ? pack_f16x2(e0, e1) : pack_bf16x2(e0, e1);
+        }
       }
       // The previous PV read P^T and wrote O^T: wait for it before both.
       if (i > 0) {
@@ -623,25 +673,48 @@ __global__ void __launch_bounds__(kF8 ? kDecThreads8 : kDecThreads, (kF8 && kR >
       // A slot that holds no token (never written, or past this sequence's
       // C slots) may hold any bits, NaN included, and its V row is still
       // multiplied by P = 0: its row of the V operand is zeroed.
-      if (!kF8 && __any_sync(0xffffffffu, pos < 0)) {
+      if ((!kF8 || kPv8) && __any_sync(0xffffffffu, pos < 0)) {
         const int sv = i % kStages;
         ok = __all_sync(0xffffffffu, mbar_wait(&ctl->v_full[sv], (i / kStages) & 1, abort, &g_device_error,
                                                kDevErrTimeoutDecode));
         if (!ok) continue;
         if (pos < 0) {
-          uint4* vrow = reinterpret_cast<uint4*>(sV + sv * kDecKvBytes + (kl >> 3) * 1024 + (kl & 7) * 128);
+          if constexpr (kPv8) {
+            // e4m3 bytes: the slot's 64-byte row (its chunks permuted within it)
+            uint4* vrow = reinterpret_cast<uint4*>(sV + sv * kTileB + kl * kHeadDim);
 #pragma unroll
-          for (int c = 0; c < 8; ++c) vrow[c] = make_uint4(0u, 0u, 0u, 0u);
+            for (int c = 0; c < 4; ++c) vrow[c] = make_uint4(0u, 0u, 0u, 0u);
+          } else {
+            uint4* vrow = reinterpret_cast<uint4*>(sV + sv * kDecKvBytes + (kl >> 3) * 1024 + (kl & 7) * 128);
+#pragma unroll
+            for (int c = 0; c < 8; ++c) vrow[c] = make_uint4(0u, 0u, 0u, 0u);
+          }
         }
       }
-      // P^T [slot kl][rows]: 128 B per slot, 16-byte chunk c (rows 8c..8c+7)
-      // at chunk position c ^ (kl % 8).
-      uint8_t* line = sP + (kl >> 3) * 1024 + (kl & 7) * 128;
+      if constexpr (kPv8) {
+        // P^T [slot kl][rows] in e4m3: 64 B per slot, 16-byte chunk c (rows
+        // 16c..16c+15) at chunk position c ^ ((kl >> 1) & 3) (64-byte swizzle).
+        uint8_t* line = sP + kl * kDecRows;
+        if constexpr (kR == 8) {
+          *reinterpret_cast<uint2*>(line + ((0 ^ ((kl >> 1) & 3)) << 4)) = make_uint2(pk[0], pk[1]);
+        } else {
 #pragma unroll
-      for (int c = 0; c < kR / 8; ++c) {
-        if (c * 8 < p.R)
-          *reinterpret_cast<uint4*>(line + ((c ^ (kl & 7)) << 4)) =
-              make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+          for (int c = 0; c < kR / 16; ++c) {
+            if (c * 16 < p.R)
+              *reinterpret_cast<uint4*>(line + ((c ^ ((kl >> 1) & 3)) << 4)) =
+                  make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+          }
+        }
+      } else {
+        // P^T [slot kl][rows]: 128 B per slot, 16-byte chunk c (rows 8c..8c+7)
+        // at chunk position c ^ (kl % 8).
+        uint8_t* line = sP + (kl >> 3) * 1024 + (kl & 7) * 128;
+#pragma unroll
+        for (int c = 0; c < kR / 8; ++c) {
+          if (c * 8 < p.R)
+            *reinterpret_cast<uint4*>(line + ((c ^ (kl & 7)) << 4)) =
+                make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+        }
       }
       fence_proxy_async_smem();
       tc_fence_before();

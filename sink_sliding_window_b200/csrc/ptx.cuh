@@ -215,6 +215,18 @@ __device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_
       : "memory");
 }
 
+// D(tmem) (+)= A(smem) * B(smem); kind::f8f6f4 (8-bit A and B as the
+// instruction descriptor's formats say, fp32 accumulate; K = 32 per MMA).
+__device__ __forceinline__ void mma_ss_f8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // D(tmem) (+)= A(tmem) * B(smem); A is K-major in TMEM (two bf16 per column).
 __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
                                        uint32_t accumulate) {
@@ -258,6 +270,30 @@ __device__ __forceinline__ uint64_t make_sdesc_sw128(uint32_t smem_addr, uint32_
   d |= uint64_t((sbo_bytes >> 4) & 0x3FFFu) << 32;
   d |= uint64_t(1) << 46;
   d |= uint64_t(2) << 61;
+  return d;
+}
+
+// Instruction descriptor, kind::f8f6f4 with e4m3 A and B (format fields 0)
+// and fp32 D: the same fields as make_idesc_f16.
+__host__ __device__ constexpr uint32_t make_idesc_e4m3(int M, int N, int a_mn_major, int b_mn_major) {
+  return (1u << 4) | (uint32_t(a_mn_major) << 15) | (uint32_t(b_mn_major) << 16) | (uint32_t(N >> 3) << 17) |
+         (uint32_t(M >> 4) << 24);
+}
+
+// Shared-memory matrix descriptor for a 64-byte-swizzled tile (the layout a
+// TMA load with CU_TENSOR_MAP_SWIZZLE_64B writes into a 512-byte aligned
+// buffer: 16-byte chunk c of 64-byte row r at chunk c ^ ((r >> 1) & 3)); swizzle
+// mode field 4.  For an 8-bit MN-major operand: rows of 64 MN-elements, one
+// per K index, at 64-byte pitch; SBO = 512 (the next group of 8 K indices);
+// LBO = the distance to the next 64-element MN group.  Advancing K by 32
+// elements adds 2048 bytes.
+__device__ __forceinline__ uint64_t make_sdesc_sw64(uint32_t smem_addr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+  uint64_t d = 0;
+  d |= uint64_t((smem_addr & 0x3FFFFu) >> 4);
+  d |= uint64_t((lbo_bytes >> 4) & 0x3FFFu) << 16;
+  d |= uint64_t((sbo_bytes >> 4) & 0x3FFFu) << 32;
+  d |= uint64_t(1) << 46;
+  d |= uint64_t(4) << 61;
   return d;
 }
 

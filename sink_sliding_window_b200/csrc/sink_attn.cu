@@ -367,10 +367,12 @@ int sink_attn_decode_launches(const sink_attn_decode_dims* d, int window) {
 
 namespace {
 
+// mode: 0 bf16 cache; 1 e4m3 cache, fp16 MMAs; 2 e4m3 cache, FP8 PV.
 sink_attn_status decode_impl(const sink_attn_decode_dims* d, const void* q, const void* k_new, const void* v_new,
                              void* k_cache, void* v_cache, const int* cache_seqlens, const float* k_scale,
-                             const float* v_scale, bool e4m3, const float* sinks, int window, float scale, void* out,
+                             const float* v_scale, int mode, const float* sinks, int window, float scale, void* out,
                              float* lse, void* workspace, size_t workspace_bytes, void* stream) {
+  const bool e4m3 = mode != 0;
   DecPlan plan;
   sink_attn_status st = plan_decode(d, window, scale, &plan);
   if (st != SINK_ATTN_OK) return st;
@@ -409,16 +411,18 @@ sink_attn_status decode_impl(const sink_attn_decode_dims* d, const void* q, cons
   }
   // Register arrays sized for the real query rows.
   using Kern = void (*)(CUtensorMap, CUtensorMap, CUtensorMap, DecParams);
-  static const Kern kerns[2][4] = {
-      {sink_attn_decode_kernel<8, false>, sink_attn_decode_kernel<16, false>, sink_attn_decode_kernel<32, false>,
-       sink_attn_decode_kernel<64, false>},
-      {sink_attn_decode_kernel<8, true>, sink_attn_decode_kernel<16, true>, sink_attn_decode_kernel<32, true>,
-       sink_attn_decode_kernel<64, true>}};
-  static SmemAttrOnce smem_set[2][4];
+  static const Kern kerns[3][4] = {
+      {sink_attn_decode_kernel<8, 0>, sink_attn_decode_kernel<16, 0>, sink_attn_decode_kernel<32, 0>,
+       sink_attn_decode_kernel<64, 0>},
+      {sink_attn_decode_kernel<8, 1>, sink_attn_decode_kernel<16, 1>, sink_attn_decode_kernel<32, 1>,
+       sink_attn_decode_kernel<64, 1>},
+      {sink_attn_decode_kernel<8, 2>, sink_attn_decode_kernel<16, 2>, sink_attn_decode_kernel<32, 2>,
+       sink_attn_decode_kernel<64, 2>}};
+  static SmemAttrOnce smem_set[3][4];
   const int vi = p.R <= 8 ? 0 : (p.R <= 16 ? 1 : (p.R <= 32 ? 2 : 3));
-  const Kern kern = kerns[e4m3][vi];
-  const size_t smem = e4m3 ? kDecSmemBytes8 : kDecSmemBytes;
-  if (!smem_set[e4m3][vi].ensure(kern, smem)) return SINK_ATTN_ERR_CUDA;
+  const Kern kern = kerns[mode][vi];
+  const size_t smem = mode == 2 ? kDecSmemBytesPv8 : (mode == 1 ? kDecSmemBytes8 : kDecSmemBytes);
+  if (!smem_set[mode][vi].ensure(kern, smem)) return SINK_ATTN_ERR_CUDA;
   const long long ctas = static_cast<long long>(p.batch) * p.Hkv * p.n_split;
   if (ctas > 0x7fffffff) return SINK_ATTN_ERR_UNSUPPORTED;
 
@@ -451,7 +455,7 @@ sink_attn_status sink_attn_decode(const sink_attn_decode_dims* d, const void* q,
                                   const void* v_new, void* k_cache, void* v_cache, const int* cache_seqlens,
                                   const float* sinks, int window, float scale, void* out, float* lse,
                                   void* workspace, size_t workspace_bytes, void* stream) {
-  return decode_impl(d, q, k_new, v_new, k_cache, v_cache, cache_seqlens, nullptr, nullptr, false, sinks, window,
+  return decode_impl(d, q, k_new, v_new, k_cache, v_cache, cache_seqlens, nullptr, nullptr, 0, sinks, window,
                      scale, out, lse, workspace, workspace_bytes, stream);
 }
 
@@ -460,7 +464,16 @@ sink_attn_status sink_attn_decode_e4m3(const sink_attn_decode_dims* d, const voi
                                        const float* k_scale, const float* v_scale, const float* sinks, int window,
                                        float scale, void* out, float* lse, void* workspace, size_t workspace_bytes,
                                        void* stream) {
-  return decode_impl(d, q, k_new, v_new, k_cache, v_cache, cache_seqlens, k_scale, v_scale, true, sinks, window,
+  return decode_impl(d, q, k_new, v_new, k_cache, v_cache, cache_seqlens, k_scale, v_scale, 1, sinks, window,
+                     scale, out, lse, workspace, workspace_bytes, stream);
+}
+
+sink_attn_status sink_attn_decode_e4m3_f8pv(const sink_attn_decode_dims* d, const void* q, const void* k_new,
+                                            const void* v_new, void* k_cache, void* v_cache,
+                                            const int* cache_seqlens, const float* k_scale, const float* v_scale,
+                                            const float* sinks, int window, float scale, void* out, float* lse,
+                                            void* workspace, size_t workspace_bytes, void* stream) {
+  return decode_impl(d, q, k_new, v_new, k_cache, v_cache, cache_seqlens, k_scale, v_scale, 2, sinks, window,
                      scale, out, lse, workspace, workspace_bytes, stream);
 }
 

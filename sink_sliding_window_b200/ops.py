@@ -28,7 +28,7 @@ STATUS = {
 EXPORTS = ("sink_attn_fwd", "sink_attn_bwd", "sink_attn_bwd_workspace_size", "sink_attn_status_string",
            "sink_attn_last_device_error", "sink_attn_device_error", "sink_attn_fwd_launches", "sink_attn_bwd_launches", "sink_attn_profile_events",
            "sink_attn_decode", "sink_attn_decode_workspace_size", "sink_attn_decode_launches",
-           "sink_attn_decode_e4m3", "sink_attn_selftest_wait")
+           "sink_attn_decode_e4m3", "sink_attn_decode_e4m3_f8pv", "sink_attn_selftest_wait")
 
 
 class SinkAttnError(RuntimeError):
@@ -87,6 +87,8 @@ def load():
         L.sink_attn_decode_e4m3.argtypes = [DD, P, P, P, P, P, P, P, P, P, I, ctypes.c_float, P, P, P,
                                             ctypes.c_size_t, P]
         L.sink_attn_decode_e4m3.restype = I
+        L.sink_attn_decode_e4m3_f8pv.argtypes = L.sink_attn_decode_e4m3.argtypes
+        L.sink_attn_decode_e4m3_f8pv.restype = I
         L.sink_attn_decode_workspace_size.argtypes = [DD, I]
         L.sink_attn_decode_workspace_size.restype = ctypes.c_size_t
         L.sink_attn_decode_launches.argtypes = [DD, I]
@@ -231,10 +233,11 @@ def decode(q, k_new, v_new, k_cache, v_cache, cache_seqlens, sinks, window=0, sc
 
 
 def decode_e4m3(q, k_new, v_new, k_cache, v_cache, cache_seqlens, k_scale, v_scale, sinks, window=0, scale=None, *,
-                max_seqlen=None, out=None, lse=None, workspace=None, stream=None):
+                max_seqlen=None, out=None, lse=None, workspace=None, stream=None, f8pv=False):
     """sink_attn_decode_e4m3: as decode(), with k_cache / v_cache holding e4m3
     codes ([B, C, Hkv, D] uint8 or torch.float8_e4m3fn) and k_scale / v_scale
-    fp32 [Hkv] dequantisation scales."""
+    fp32 [Hkv] dequantisation scales.  f8pv: sink_attn_decode_e4m3_f8pv (the
+    PV product in FP8, P rounded to e4m3)."""
     B, Lq, Hq, D = q.shape
     C, Hkv = k_cache.shape[1], k_cache.shape[2]
     if max_seqlen is None:
@@ -250,13 +253,19 @@ def decode_e4m3(q, k_new, v_new, k_cache, v_cache, cache_seqlens, k_scale, v_sca
     if workspace is None:
         need = int(L.sink_attn_decode_workspace_size(ctypes.byref(dims), int(window)))
         workspace = torch.empty((max(need, 1),), dtype=torch.uint8, device=q.device)
-    st = L.sink_attn_decode_e4m3(ctypes.byref(dims), _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_cache),
-                                 _ptr(v_cache), _ptr(cache_seqlens), _ptr(k_scale), _ptr(v_scale), _ptr(sinks),
-                                 int(window), float(scale), _ptr(out), _ptr(lse), _ptr(workspace),
-                                 ctypes.c_size_t(workspace.numel()), _stream_handle(stream))
+    fn, name = ((L.sink_attn_decode_e4m3_f8pv, "sink_attn_decode_e4m3_f8pv") if f8pv
+                else (L.sink_attn_decode_e4m3, "sink_attn_decode_e4m3"))
+    st = fn(ctypes.byref(dims), _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache), _ptr(cache_seqlens),
+            _ptr(k_scale), _ptr(v_scale), _ptr(sinks), int(window), float(scale), _ptr(out), _ptr(lse),
+            _ptr(workspace), ctypes.c_size_t(workspace.numel()), _stream_handle(stream))
     if st != 0:
-        raise SinkAttnError(st, "sink_attn_decode_e4m3")
+        raise SinkAttnError(st, name)
     return out, lse
+
+
+def decode_e4m3_f8pv(*args, **kw):
+    """sink_attn_decode_e4m3_f8pv (see decode_e4m3)."""
+    return decode_e4m3(*args, f8pv=True, **kw)
 
 
 def device_error(stream=None) -> int:

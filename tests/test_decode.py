@@ -154,7 +154,46 @@ def test_launch_count(ops):
 
 
 # ----------------------------------------------------------------- e4m3 cache
-def _run_e4m3(ops, cached, Lq, Hq, Hkv, C, window, seed, seqs=None, heavy=False):
+def _f8pv_bounds(qd, kd, vd, sinks, cu, cached, Lq, window, seqs, ro, rl):
+    """Per-element bounds for the FP8 PV variant, from the definition and the
+    e4m3 format.  The kernel rounds each unnormalised weight p_j = 2^(x_j - m)
+    (m its running reference, with 1 <= max(p, sink term) <= 2^8 and so
+    Z = sum p + sink term >= 1) to e4m3: |p~ - p| <= 2^-4 p in e4m3's normal
+    range (p >= 2^-6) and <= 2^-10 below it.  With the same p~ in the row
+    sums, out~ - out = sum_j (p~_j - p_j)(v_j - out) / Z~, hence (pi_j =
+    p_j / Z, the normalised weights; 1 / Z <= pi_max):
+      |out~ - out| <= 2^-4 sum_j pi_j |v_j - out| + 2^-10 pi_max sum_j |v_j - out|
+      |lse~ - lse| <= 2^-4 sum_j pi_j + 2^-10 pi_max N.
+    Returns (out bound [rows, Hq, D], lse bound [Hq, rows]) for the rows of
+    `seqs` in the order of ro / rl."""
+    Hq = qd.shape[2]
+    G = Hq // kd.shape[1]
+    ob, lb = [], []
+    r = 0
+    for b in seqs:
+        lo = int(cu[b])
+        for t in range(Lq):
+            pos = int(cached[b]) + t
+            j0 = max(0, pos - window + 1) if window > 0 else 0
+            K = kd[lo + j0:lo + pos + 1]  # [N, Hkv, D]
+            V = vd[lo + j0:lo + pos + 1]
+            ob_r = np.zeros((Hq, kd.shape[2]))
+            for h in range(Hq):
+                g = h // G
+                logits = SCALE * (K[:, g] @ qd[b, t, h])
+                pi = np.exp(logits - rl[h, r])
+                dev_ = np.abs(V[:, g] - ro[r, h][None, :])  # [N, D]
+                ob_r[h] = 2.0 ** -4 * (pi[:, None] * dev_).sum(0) + 2.0 ** -10 * pi.max() * dev_.sum(0)
+                lb.append((h, r, 2.0 ** -4 * pi.sum() + 2.0 ** -10 * pi.max() * len(pi)))
+            ob.append(ob_r)
+            r += 1
+    lbound = np.zeros((Hq, r))
+    for h, rr, v in lb:
+        lbound[h, rr] = v
+    return np.stack(ob), lbound
+
+
+def _run_e4m3(ops, cached, Lq, Hq, Hkv, C, window, seed, seqs=None, heavy=False, f8pv=False):
     """The e4m3-cache decode: history tokens enter the cache as host-quantised
     codes (per-head scale = amax / 448), the new tokens are quantised by the
     call.  The oracle gets the dequantised values code * scale exactly (fp64),
@@ -193,9 +232,9 @@ def _run_e4m3(ops, cached, Lq, Hq, Hkv, C, window, seed, seqs=None, heavy=False)
     k_new = a["k"][new_idx].reshape(B, Lq, Hkv, 64)
     v_new = a["v"][new_idx].reshape(B, Lq, Hkv, 64)
     kc, vc = torch.from_numpy(kc0).cuda(), torch.from_numpy(vc0).cuda()
-    out, lse = ops.decode_e4m3(dev_bf16(a["q_new"]), dev_bf16(k_new), dev_bf16(v_new), kc, vc,
-                               dev(np.asarray(cached, np.int32)), dev(ks), dev(vs), dev(a["sinks"]), window, SCALE,
-                               max_seqlen=int(max(cached)) + Lq)
+    call = ops.decode_e4m3_f8pv if f8pv else ops.decode_e4m3
+    out, lse = call(dev_bf16(a["q_new"]), dev_bf16(k_new), dev_bf16(v_new), kc, vc, dev(np.asarray(cached, np.int32)),
+                    dev(ks), dev(vs), dev(a["sinks"]), window, SCALE, max_seqlen=int(max(cached)) + Lq)
     torch.cuda.synchronize()
     assert ops.device_error() == 0
     ke, ve = kc0.copy(), vc0.copy()
@@ -222,8 +261,23 @@ def _run_e4m3(ops, cached, Lq, Hq, Hkv, C, window, seed, seqs=None, heavy=False)
         lses.append(l)
     got_o = host_f64(out)[seqs].reshape(-1, Hq, 64)
     got_l = host_f64(lse).reshape(Hq, B, Lq)[:, seqs].reshape(Hq, -1)
-    check(got_o, np.concatenate(outs), TOL_OUT, "e4m3 decode out")
-    check(got_l, np.concatenate(lses, axis=1), TOL_LSE, "e4m3 decode lse")
+    ro, rl = np.concatenate(outs), np.concatenate(lses, axis=1)
+    if not f8pv:
+        check(got_o, ro, TOL_OUT, "e4m3 decode out")
+        check(got_l, rl, TOL_LSE, "e4m3 decode lse")
+        return
+    # FP8 PV: P is rounded to e4m3 before the MMA; the bound of that rounding
+    # (_f8pv_bounds) plus the usual budget for the other roundings.
+    qd_new = qd.reshape(B, Lq, Hq, 64)
+    ob, lb = _f8pv_bounds(qd_new, kd, vd, a["sinks"], cu, cached, Lq, window, seqs, ro, rl)
+    assert np.all(np.isfinite(got_o)) and np.all(np.isfinite(got_l)), "FP8 PV decode: non-finite values"
+    eo = np.abs(got_o - ro)
+    assert np.all(eo <= 1.05 * ob + TOL_OUT * np.abs(ro).max()), \
+        f"FP8 PV decode out beyond its bound: worst excess {np.max(eo - 1.05 * ob - TOL_OUT * np.abs(ro).max()):.3e}"
+    el = np.abs(got_l - rl)
+    assert np.all(el <= 1.05 * lb + TOL_LSE * np.abs(rl).max()), \
+        f"FP8 PV decode lse beyond its bound: worst excess {np.max(el - 1.05 * lb - TOL_LSE * np.abs(rl).max()):.3e}"
+    print(f"FP8 PV decode: out error {eo.max():.3e} (bound max {ob.max():.3e}), lse error {el.max():.3e}")
 
 
 @pytest.mark.parametrize("window,C,Lq", [(0, 1152, 1), (100, 1152, 1), (128, 128, 1), (128, 129, 2), (16, 18, 3)])
@@ -250,3 +304,25 @@ def test_e4m3_cache_gpt_oss_full_size(ops, window, C):
     ring fits one CTA per (sequence, key/value head), which then finishes
     the rows itself (no combine launch)."""
     _run_e4m3(ops, [8191] * 62 + [0, 4000], 1, 64, 8, C, window, seed=80, seqs=[0, 31, 62, 63])
+
+
+# -------------------------------------------- e4m3 cache, FP8 PV product
+@pytest.mark.parametrize("window,C,Lq", [(0, 1152, 1), (100, 1152, 1), (128, 128, 1), (128, 129, 2), (16, 18, 3)])
+def test_e4m3_f8pv(ops, window, C, Lq):
+    """sink_attn_decode_e4m3_f8pv: the PV product on the FP8 tensor-core path
+    (P rounded to e4m3), against the oracle within the bound that rounding
+    implies; the cache after append is checked bit for bit."""
+    _run_e4m3(ops, [0, 1, 99, 127, 128, 129, 300, 1000], Lq, 16, 2, C, window, seed=160 + Lq, f8pv=True)
+
+
+@pytest.mark.parametrize("G,Lq", [(1, 1), (8, 1), (8, 4), (16, 4)])
+def test_e4m3_f8pv_row_variants(ops, G, Lq):
+    """Every register-tile variant (8, 16, 32, 64 query rows)."""
+    _run_e4m3(ops, [0, 64, 257], Lq, 2 * G, 2, 512, 0, seed=170 + G, f8pv=True)
+
+
+@pytest.mark.parametrize("window,C", [(0, 8192), (128, 128)])
+def test_e4m3_f8pv_gpt_oss_full_size(ops, window, C):
+    """gpt-oss heads, 64 sequences at 8191 cached tokens + 1 (split and
+    combined on the 8192-slot cache; one CTA per head group on the ring)."""
+    _run_e4m3(ops, [8191] * 62 + [0, 4000], 1, 64, 8, C, window, seed=180, seqs=[0, 31, 62, 63], f8pv=True)
