@@ -38,6 +38,8 @@ from sink_sliding_window_b200 import synth  # noqa: E402
 WORKLOAD = "prefill4k"
 B, S, HQ, HKV, D = 4, 4096, 64, 8, 64
 LAYERS = (128, 0)  # window per layer: sliding window 128, then full causal
+# The forward kernels timed one by one next to sink_attn_fwd's own choice.
+FWD_KERNEL_NAMES = ("one_tile", "two_tiles", "pair")
 METRIC = "sink-attn fwd/bwd TFLOP/s (unmasked FLOPs) and % of B200 bf16 tensor peak"
 
 
@@ -175,13 +177,17 @@ def read_peaks():
     return 1590.0, 6650.0, "fallback"
 
 
+# Sources the backward main kernel is compiled from (its measured DRAM
+# traffic is reported only while these are unchanged).
+BWD_MAIN_SOURCES = ("bwd_kernels.cuh", "common.cuh", "ptx.cuh", "tmem_io.cuh", "tma_host.cuh")
+
+
 def kernel_source_hash():
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "sink_sliding_window_b200", "csrc")
-    for n in sorted(os.listdir(csrc)):
-        if n.endswith((".cu", ".cuh")):
-            with open(os.path.join(csrc, n), "rb") as f:
-                h.update(n.encode() + f.read())
+    for n in BWD_MAIN_SOURCES:
+        with open(os.path.join(csrc, n), "rb") as f:
+            h.update(n.encode() + f.read())
     return h.hexdigest()[:16]
 
 
@@ -291,6 +297,10 @@ def measure_layers(torch, ops, stream, q, k, v, sinks, dout, outs, grads, ws, it
                                     workspace=ws, **kw),
                     nb(q, k, v, sinks, o, l, dout) + nb(dq, dk, dv, ds)),
         }
+        for kn in FWD_KERNEL_NAMES:
+            calls["fwd:" + kn] = ((lambda kn=kn: ops.fwd(q, k, v, sinks, None, W, 0.125, out=o, lse=l, kernel=kn,
+                                                         **kw)),
+                                  calls["fwd"][1])
         fl = dict(zip(("fwd", "bwd"), layer_flops(W)))
         entry = {"window": W, "workload": f"{WORKLOAD} ({'window %d' % W if W > 0 else 'full causal'})"}
         for name, (fn, min_bytes) in calls.items():
@@ -304,8 +314,13 @@ def measure_layers(torch, ops, stream, q, k, v, sinks, dout, outs, grads, ws, it
             e1.record(stream)
             torch.cuda.synchronize()
             ms = e0.elapsed_time(e1) / iters
-            entry[name] = {"ms": ms, "tflops": fl[name] / ms / 1e9, "min_bytes": min_bytes,
-                           "GBps": min_bytes / ms / 1e6, "hbm_frac": min_bytes / ms / 1e6 / hbm}
+            r = {"ms": ms, "tflops": fl[name.split(":")[0]] / ms / 1e9, "min_bytes": min_bytes,
+                 "GBps": min_bytes / ms / 1e6, "hbm_frac": min_bytes / ms / 1e6 / hbm}
+            if ":" in name:
+                entry.setdefault("fwd_kernels", {})[name.split(":")[1]] = r
+            else:
+                entry[name] = r
+        entry["fwd"]["kernel"] = ops.fwd_kernel_for(T, HQ, HKV, D, B, S, W)
         entry["peak_GBps"] = hbm
         entry["peak_source"] = f"{kind} hbm_gbs"
         res.append(entry)
@@ -341,7 +356,8 @@ def layer_calls(ops, w, t, stream, window, bufs):
         kw = dict(batch=w.batch, max_seqlen=w.uniform_seqlen, stream=stream)
     else:
         kw = dict(max_seqlen=w.max_seqlen, stream=stream)
-    f = lambda: ops.fwd(t["q"], t["k"], t["v"], t["sinks"], t["cu"], window, w.scale, out=o, lse=l, **kw)  # noqa
+    f = lambda kernel="auto": ops.fwd(t["q"], t["k"], t["v"], t["sinks"], t["cu"], window, w.scale,  # noqa
+                                      out=o, lse=l, kernel=kernel, **kw)
     b = lambda: ops.bwd(t["q"], t["k"], t["v"], t["sinks"], o, l, t["dout"], t["cu"], window, w.scale, dq=dq,  # noqa
                         dk=dk, dv=dv, dsinks=ds, workspace=ws, **kw)
     return f, b
@@ -378,9 +394,11 @@ def measure_extra(torch, ops, stream, iters=5):
             f, b = layer_calls(ops, w, t, stream, window, bufs)
             p = pairs(w.cu_seqlens, window, w.Hq)
             lay = {"window": window}
-            for name, fn, flops, mb in (
-                    ("fwd", f, 4 * D * p, nb(t["q"], t["k"], t["v"], t["sinks"], o, l)),
-                    ("bwd", b, 10 * D * p, nb(t["q"], t["k"], t["v"], t["sinks"], o, l, t["dout"], dq, dk, dv, ds))):
+            fwd_mb = nb(t["q"], t["k"], t["v"], t["sinks"], o, l)
+            cases = [("fwd", f, 4 * D * p, fwd_mb)]
+            cases += [("fwd:" + kn, (lambda kn=kn: f(kn)), 4 * D * p, fwd_mb) for kn in FWD_KERNEL_NAMES]
+            cases += [("bwd", b, 10 * D * p, nb(t["q"], t["k"], t["v"], t["sinks"], o, l, t["dout"], dq, dk, dv, ds))]
+            for name, fn, flops, mb in cases:
                 for _ in range(2):
                     fn()
                 torch.cuda.synchronize()
@@ -391,8 +409,13 @@ def measure_extra(torch, ops, stream, iters=5):
                 e1.record(stream)
                 torch.cuda.synchronize()
                 ms = e0.elapsed_time(e1) / iters
-                lay[name] = {"ms": ms, "tflops": flops / ms / 1e9, "pct_of_peak": 100.0 * flops / ms / 1e9 / peak,
-                             "min_bytes": mb, "GBps": mb / ms / 1e6, "hbm_frac": mb / ms / 1e6 / hbm}
+                r = {"ms": ms, "tflops": flops / ms / 1e9, "pct_of_peak": 100.0 * flops / ms / 1e9 / peak,
+                     "min_bytes": mb, "GBps": mb / ms / 1e6, "hbm_frac": mb / ms / 1e6 / hbm}
+                if ":" in name:
+                    lay.setdefault("fwd_kernels", {})[name.split(":")[1]] = r
+                else:
+                    lay[name] = r
+            lay["fwd"]["kernel"] = ops.fwd_kernel_for(w.T, w.Hq, w.Hkv, w.D, w.batch, w.max_seqlen, window)
             entry["layers"].append(lay)
         entry["peak_TFLOPs"], entry["peak_GBps"], entry["peak_source"] = peak, hbm, f"{kind} bf16_tflops / hbm_gbs"
         res[base] = entry
@@ -404,13 +427,16 @@ def measure_extra(torch, ops, stream, iters=5):
 
 
 def run_profile_case(args):
-    """--profile-case KIND:WORKLOAD:LAYER (e.g. fwd:long60k:full,
-    bwd:prefill4k:w128): two calls of one entry point on one workload, for an
+    """--profile-case KIND:WORKLOAD:LAYER (e.g. fwd:long60k:full, fwd.pair:long60k:full,
+    fwd.two_tiles:prefill4k:w128, bwd:prefill4k:w128; fwd.<kernel> runs one of
+    the forward kernels explicitly): two calls of one entry point on one workload, for an
     ncu capture of its kernels (capture the second: -s <launches of one
     call>).  Prints nothing but a done line."""
     import torch
     from sink_sliding_window_b200 import build, ops
     kind, name = args.profile_case.split(":", 1)
+    kind, _, fwd_kernel = kind.partition(".")
+    fwd_kernel = fwd_kernel or "auto"
     torch.cuda.set_device(0)
     build.build()
     ops.load()
@@ -422,7 +448,10 @@ def run_profile_case(args):
     if kind == "bwd":
         f()
     for _ in range(2):
-        (f if kind == "fwd" else b)()
+        if kind == "fwd":
+            f(fwd_kernel)
+        else:
+            b()
     torch.cuda.synchronize()
     if ops.device_error() != 0:
         raise RuntimeError("a kernel reported a timed-out wait")

@@ -93,6 +93,53 @@ sink_attn_status sink_attn_fwd(const sink_attn_dims* dims,
                                int window, float scale,
                                void* out, float* lse, void* stream);
 
+/* Forward on CTA pairs: the same operation, arguments, layouts, ownership
+ * and errors as sink_attn_fwd() (the online softmax with the sink logit as
+ * the first reference max, "Tricks from OpenAI gpt-oss you can use with
+ * transformers", kernels section; the window and document masks of "gpt-oss
+ * implementation", alternating sliding-window pattern), computed by a kernel
+ * launched as clusters of two CTAs whose tensor-core MMAs run on the CTA
+ * pair (M = 256 rows: two adjacent query tiles of one key/value head).  Each
+ * CTA loads half of every key and value step, and one thread issues the
+ * pair's MMAs.  The two tiles of a pair walk the union of their key ranges,
+ * so a row's keys may be split into 64-key steps at other boundaries than
+ * in sink_attn_fwd(): the results agree with it to rounding, not bit for
+ * bit.  Returns SINK_ATTN_ERR_CUDA if the device cannot run clusters of two
+ * CTAs of this kernel. */
+sink_attn_status sink_attn_fwd_pair(const sink_attn_dims* dims,
+                                    const void* q, const void* k, const void* v,
+                                    const float* sinks, const int* cu_seqlens,
+                                    int window, float scale,
+                                    void* out, float* lse, void* stream);
+
+/* The forward kernels of this library.  All compute the same operation with
+ * the same arguments; they differ in how query tiles (128 rows: 128/G tokens
+ * x the G query heads of one key/value head) map to CTAs, and their results
+ * agree to rounding, not bit for bit, because a row's keys may be split into
+ * 64-key steps at other boundaries. */
+typedef enum {
+    SINK_ATTN_FWD_AUTO = 0,      /* the kernel sink_attn_fwd() picks for the sizes */
+    SINK_ATTN_FWD_ONE_TILE = 1,  /* one query tile per CTA; its two softmax warpgroups take alternate
+                                    64-key steps and merge at the end */
+    SINK_ATTN_FWD_TWO_TILES = 2, /* two adjacent query tiles per CTA, one per softmax warpgroup, sharing
+                                    one key/value stream (short key ranges: sliding-window layers) */
+    SINK_ATTN_FWD_CTA_PAIR = 3   /* two adjacent query tiles on a pair of CTAs (cluster of two) with
+                                    M = 256 tensor-core MMAs, as sink_attn_fwd_pair() */
+} sink_attn_fwd_kernel_id;
+
+/* The forward with an explicit kernel (a sink_attn_fwd_kernel_id); arguments,
+ * layouts and errors as sink_attn_fwd().  An unknown id returns
+ * SINK_ATTN_ERR_UNSUPPORTED before any launch. */
+sink_attn_status sink_attn_fwd_with(const sink_attn_dims* dims,
+                                    const void* q, const void* k, const void* v,
+                                    const float* sinks, const int* cu_seqlens,
+                                    int window, float scale,
+                                    void* out, float* lse, int kernel, void* stream);
+
+/* The sink_attn_fwd_kernel_id sink_attn_fwd() runs for these sizes and
+ * window (never SINK_ATTN_FWD_AUTO), or -1 when the sizes are invalid. */
+int sink_attn_fwd_kernel_for(const sink_attn_dims* dims, int window);
+
 /* Bytes of device workspace sink_attn_bwd() needs for these sizes
  * (fp32 dq accumulator, per-row D_i, per-block sink partials, padding).
  * Returns 0 when the sizes are invalid. */

@@ -259,7 +259,7 @@ struct BwdCtl {
 // with the same bounded wait as every other wait in these kernels.
 __device__ __forceinline__ bool group_sync(uint64_t* bar, uint32_t& phase, volatile int* abort, int code) {
   mbar_arrive(bar);
-  const bool ok = mbar_wait(bar, phase, abort, &g_device_error, code);
+  const bool ok = warp_all(mbar_wait(bar, phase, abort, &g_device_error, code));
   phase ^= 1u;
   return ok;
 }
@@ -534,6 +534,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const uint32_t sbuf = (i & 1) ? kBwdTmemS1 : kBwdTmemS0;
       ok = mbar_wait(&ctl->qdo_full[st], (i / kBwdStages) & 1, abort, &g_device_error, kDevErrTimeoutSoftmax) &&
            mbar_wait(&ctl->s_full[i & 1], (i >> 1) & 1, abort, &g_device_error, kDevErrTimeoutSoftmax);
+      ok = warp_all(ok);
       if (!ok) break;
       tc_fence_after();
       const BwdAux& a = aux[st];
@@ -558,7 +559,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       // this warp has read them and no other warp reads them.
       __syncwarp();
       tmem_st32_nowait(tmem + lane_base + sbuf + 64 * ch, pk);
-      ok = mbar_wait(&ctl->dp_full, i & 1, abort, &g_device_error, kDevErrTimeoutSoftmax);
+      ok = warp_all(mbar_wait(&ctl->dp_full, i & 1, abort, &g_device_error, kDevErrTimeoutSoftmax));
       if (!ok) break;
       tc_fence_after();
       // dS = P (dP - D); dQ_{i-1} has finished reading the shared dS buffer
@@ -608,6 +609,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
     // ------------------------------------------ dK (ch 0) / dV (ch 1) epilogue
     if (ok) ok = mbar_wait(&ctl->kd_full, 0, abort, &g_device_error, kDevErrTimeoutEpilogue);
+    ok = warp_all(ok);
     if (ok) {
       tc_fence_after();
       uint32_t r[kHeadDim];
@@ -637,7 +639,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     uint32_t sync_phase = 0;
     bool ok = true;
     for (int i = 0; i < w.nq; ++i) {
-      ok = mbar_wait(&ctl->dq_full, i & 1, abort, &g_device_error, kDevErrTimeoutBwd);
+      ok = warp_all(mbar_wait(&ctl->dq_full, i & 1, abort, &g_device_error, kDevErrTimeoutBwd));
       if (!ok) break;
       tc_fence_after();
       uint32_t d[kHeadDim];

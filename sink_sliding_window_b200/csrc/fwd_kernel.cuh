@@ -31,6 +31,16 @@
 // Tiles outside the causal / window / document range are never visited; only
 // the edge steps apply an element mask.
 //
+// Two-tile mode (kTiles = 2, for short key ranges such as sliding-window
+// layers, where a one-tile CTA does only a few steps between its set-up and
+// its epilogue): the CTA owns two adjacent query tiles of the same head g,
+// warpgroup b takes every step of tile b (its own S/P buffer, O_b, running
+// max and sum, no merge), and one K/V stream over the union of the two
+// tiles' key ranges serves both; each warpgroup masks its own rows.  The MMA
+// issuer serves the warpgroups in turn (PV_b and S_b of the next step as soon
+// as P_b is written), so one warpgroup's exponentials overlap the other's
+// S round trip, as the alternating steps do in the one-tile mode.
+//
 // Warp roles (320 threads, 2 CTAs per SM): warps 0-7 softmax + epilogue (two
 // warpgroups), warp 8 TMA producer, warp 9 TMEM allocator + MMA issuer.
 // TMEM: S/P buffers in columns [0,64) and [64,128), O_0 in [128,192), O_1 in
@@ -77,29 +87,35 @@ struct FwdCtl {
   int abort;
 };
 
-constexpr size_t kFwdSmemBytes = 1024 /*alignment slack*/ + kTileBytes * (1 + 2 * kFwdStages) + sizeof(FwdCtl);
+// Q tiles (kTiles), then K and V stages, then the control block.
+template <int kTiles>
+constexpr size_t fwd_smem_bytes() {
+  return 1024 /*alignment slack*/ + kTileBytes * (kTiles + 2 * kFwdStages) + sizeof(FwdCtl);
+}
 
-// Query tile handled by this CTA and its key range.
+// Query tiles handled by this CTA (kTiles adjacent tiles of head g) and the
+// key range of their common step stream.
 struct FwdTile {
   int g;       // key/value head
-  int t0;      // first token of the tile
-  int t_last;  // last valid token of the tile
+  int t0;      // first token of the CTA's first tile
   int kv_lo;   // first key any row may see
-  int lo_max;  // first key the last row may see (largest over rows)
   int n_half;  // 64-key steps to visit
   int n_tiles; // 128-key K/V tiles to load
 };
 
+template <int kTiles>
 __device__ __forceinline__ FwdTile fwd_tile(const Geometry& geo) {
   FwdTile w;
   w.g = blockIdx.x % geo.Hkv;
   // Later tiles see more keys under a causal mask: hand them out first.
-  const int qb = geo.num_qblocks - 1 - static_cast<int>(blockIdx.x / geo.Hkv);
-  w.t0 = qb << geo.P_log2;
-  w.t_last = min(w.t0 + (1 << geo.P_log2) - 1, geo.T - 1);
+  const int units = (geo.num_qblocks + kTiles - 1) / kTiles;
+  const int u = units - 1 - static_cast<int>(blockIdx.x / geo.Hkv);
+  w.t0 = (u * kTiles) << geo.P_log2;
+  // first_key is non-decreasing in t: the first row has the smallest first
+  // key, the last valid token the largest key.
+  const int t_end = min(w.t0 + (kTiles << geo.P_log2) - 1, geo.T - 1);
   w.kv_lo = first_key(geo, w.t0);
-  w.lo_max = first_key(geo, w.t_last);
-  w.n_half = (w.t_last - w.kv_lo + kHalfN) / kHalfN;
+  w.n_half = (t_end - w.kv_lo + kHalfN) / kHalfN;
   w.n_tiles = (w.n_half + 1) / 2;
   return w;
 }
@@ -174,19 +190,21 @@ __device__ __forceinline__ FwdRowStep fwd_row_step(uint32_t* s, int c_lo, int c_
   return r;
 }
 
+template <int kTiles>
 __global__ void __launch_bounds__(kFwdThreads, 2)
     sink_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                          const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
+  static_assert(kTiles == 1 || kTiles == 2, "one or two query tiles per CTA");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   uint8_t* sQ = smem;
-  uint8_t* sK = smem + kTileBytes;
+  uint8_t* sK = smem + kTiles * kTileBytes;
   uint8_t* sV = sK + kFwdStages * kTileBytes;
   FwdCtl* ctl = reinterpret_cast<FwdCtl*>(sV + kFwdStages * kTileBytes);
   volatile int* abort = &ctl->abort;
   const int warp = threadIdx.x >> 5;
   const Geometry& geo = p.geo;
-  const FwdTile w = fwd_tile(geo);
+  const FwdTile w = fwd_tile<kTiles>(geo);
 
   if (threadIdx.x == 0) {
     mbar_init(&ctl->q_full, 1);
@@ -219,8 +237,10 @@ __global__ void __launch_bounds__(kFwdThreads, 2)
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
-      mbar_arrive_expect_tx(&ctl->q_full, kTileBytes);
-      tma_load_3d(sQ, &tm_q, &ctl->q_full, 0, w.g << geo.G_log2, w.t0);
+      mbar_arrive_expect_tx(&ctl->q_full, kTiles * kTileBytes);
+#pragma unroll
+      for (int u = 0; u < kTiles; ++u)
+        tma_load_3d(sQ + u * kTileBytes, &tm_q, &ctl->q_full, 0, w.g << geo.G_log2, w.t0 + (u << geo.P_log2));
       for (int j = 0; j < w.n_tiles; ++j) {
         const int s = j % kFwdStages;
         if (j >= kFwdStages &&
@@ -239,7 +259,50 @@ __global__ void __launch_bounds__(kFwdThreads, 2)
     // Order: S_0, S_1, then for every step h: O_{h%2} += P_h V_h, S_{h+2}
     // into the buffer P_h just left (tcgen05 MMAs of one thread execute in
     // order, so the PV reads P_h before S_{h+2} overwrites it).
-    if (elect_one()) {
+    if (kTiles == 2 && elect_one()) {
+      // Two tiles: warpgroup b's steps are S_b(h) -> P_b(h) -> O_b += P_b V(h)
+      // -> S_b(h+1) into the buffer P_b(h) just left (the PV, issued first,
+      // reads P_b(h) before the S MMA overwrites it).  S_0(0) and S_1(0) go
+      // out together; then the warpgroups are served in turn at every step.
+      const uint32_t tS = tmem + kFwdTmemS;
+      const uint32_t tO = tmem + kFwdTmemO;
+      bool ok = mbar_wait(&ctl->q_full, 0, abort, &g_device_error, kDevErrTimeoutMma) &&
+                mbar_wait(&ctl->k_full[0], 0, abort, &g_device_error, kDevErrTimeoutMma);
+      if (ok) {
+        tc_fence_after();
+#pragma unroll
+        for (int b = 0; b < 2; ++b) {
+          fwd_issue_qk(tS + b * kHalfN, smem_u32(sQ + b * kTileBytes), smem_u32(sK));
+          tc_commit(&ctl->s_full[b]);
+        }
+      }
+      for (int h = 0; ok && h < w.n_half; ++h) {
+        const int j = h >> 1;
+        const int s = j % kFwdStages;
+        const int hn = h + 1;
+        const int jn = hn >> 1;
+        const int sn = jn % kFwdStages;
+        ok = mbar_wait(&ctl->v_full[s], (j / kFwdStages) & 1, abort, &g_device_error, kDevErrTimeoutMma) &&
+             (hn >= w.n_half ||
+              mbar_wait(&ctl->k_full[sn], (jn / kFwdStages) & 1, abort, &g_device_error, kDevErrTimeoutMma));
+        for (int b = 0; ok && b < 2; ++b) {
+          ok = mbar_wait(&ctl->p_full[b], h & 1, abort, &g_device_error, kDevErrTimeoutMma);
+          if (!ok) break;
+          tc_fence_after();
+          fwd_issue_pv(tO + b * kHeadDim, tS + b * kHalfN, smem_u32(sV + s * kTileBytes) + (h & 1) * kHalfBytes,
+                       h > 0);
+          if (hn < w.n_half) {
+            fwd_issue_qk(tS + b * kHalfN, smem_u32(sQ + b * kTileBytes),
+                         smem_u32(sK + sn * kTileBytes) + (hn & 1) * kHalfBytes);
+            tc_commit(&ctl->s_full[b]);
+          }
+        }
+        // K/V tile j is done once both warpgroups' PVs of its second step
+        // (or of the last step) are.
+        if (ok && ((h & 1) == 1 || h == w.n_half - 1)) tc_commit(&ctl->kv_empty[s]);
+      }
+      if (ok) tc_commit(&ctl->o_full);
+    } else if (kTiles == 1 && elect_one()) {
       const uint32_t tS = tmem + kFwdTmemS;
       const uint32_t tO = tmem + kFwdTmemO;
       const uint32_t q_addr = smem_u32(sQ);
@@ -276,10 +339,15 @@ __global__ void __launch_bounds__(kFwdThreads, 2)
     }
   } else {
     // ------------------------------------------- softmax (1 row per thread)
-    const int wg = warp >> 2;  // steps h with h % 2 == wg
+    // One tile: warpgroup wg takes the steps h with h % 2 == wg.  Two tiles:
+    // warpgroup wg takes every step of tile wg.
+    const int wg = warp >> 2;
     const int r = threadIdx.x & (kBlockM - 1);
     const int G = 1 << geo.G_log2;
-    const int t = w.t0 + (r >> geo.G_log2);
+    const int tw0 = w.t0 + (kTiles == 2 ? (wg << geo.P_log2) : 0);  // first token of this warpgroup's tile
+    const bool rows = tw0 < geo.T;
+    const int lo_max = rows ? first_key(geo, min(tw0 + (1 << geo.P_log2) - 1, geo.T - 1)) : 0;
+    const int t = tw0 + (r >> geo.G_log2);
     const int h = (w.g << geo.G_log2) + (r & (G - 1));
     const bool valid = t < geo.T;
     int lo_r = 0, hi_r = -1;  // allowed keys [lo_r, hi_r]; empty for padding rows
@@ -288,27 +356,28 @@ __global__ void __launch_bounds__(kFwdThreads, 2)
       hi_r = t;
     }
     const float sink = __ldg(p.sinks + h);
-    // Both warpgroups take the sink logit as their first reference max; only
-    // warpgroup 0 counts the sink's own e^{s-m} = 1 in its sum.
+    // Every warpgroup takes the sink logit as its first reference max; the
+    // sink's own e^{s-m} = 1 is counted once per row (one tile: by warpgroup
+    // 0 only).
     float m_ref = sink * kLog2e;  // -inf when the sink is off
-    float l = (wg == 0 && sink != -INFINITY) ? 1.f : 0.f;
+    float l = ((kTiles == 2 || wg == 0) && sink != -INFINITY) ? 1.f : 0.f;
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t tS = tmem + lane_base + kFwdTmemS + wg * kHalfN;
     const uint32_t tO = tmem + lane_base + kFwdTmemO + wg * kHeadDim;
     const float sl2 = p.scale_log2;
     bool ok = true;
 
-    for (int hs = wg, i = 0; hs < w.n_half; hs += 2, ++i) {
-      ok = mbar_wait(&ctl->s_full[wg], i & 1, abort, &g_device_error, kDevErrTimeoutSoftmax);
+    for (int hs = (kTiles == 1 ? wg : 0), i = 0; hs < w.n_half; hs += 3 - kTiles, ++i) {
+      ok = warp_all(mbar_wait(&ctl->s_full[wg], i & 1, abort, &g_device_error, kDevErrTimeoutSoftmax));
       if (!ok) break;
       tc_fence_after();
       uint32_t sr[kHalfN];
       tmem_ld64(tS, sr);
       const int ks = w.kv_lo + hs * kHalfN;
-      // CTA-uniform: does any row of this step see a masked key?  Resolved
-      // once per step, not per element.
+      // Uniform over the tile: does any row of this step see a masked key?
+      // Resolved once per step, not per element.
       FwdRowStep st;
-      if (ks + kHalfN - 1 > w.t0 || ks < w.lo_max)
+      if (!rows || ks + kHalfN - 1 > tw0 || ks < lo_max)
         st = fwd_row_step<true>(sr, lo_r - ks, hi_r - ks, sl2, m_ref);
       else
         st = fwd_row_step<false>(sr, 0, 0, sl2, m_ref);
@@ -331,51 +400,77 @@ __global__ void __launch_bounds__(kFwdThreads, 2)
       mbar_arrive(&ctl->p_full[wg]);
     }
 
-    // ------------------------------------------------ merge and epilogue
-    // Each warpgroup publishes its (m, l); then warpgroup b writes output
-    // columns [32 b, 32 b + 32) of its rows from both accumulators.
     if (ok) ok = mbar_wait(&ctl->o_full, 0, abort, &g_device_error, kDevErrTimeoutEpilogue);
-    ctl->m_part[wg][r] = m_ref;
-    ctl->l_part[wg][r] = l;
-    uint32_t merge_phase = 0;
-    mbar_arrive(&ctl->merge);
-    if (ok) ok = mbar_wait(&ctl->merge, merge_phase, abort, &g_device_error, kDevErrTimeoutEpilogue);
-    if (ok) {
-      tc_fence_after();
-      const bool has1 = w.n_half >= 2;  // warpgroup 1 saw at least one step
-      const float m0 = ctl->m_part[0][r], l0 = ctl->l_part[0][r];
-      const float m1 = has1 ? ctl->m_part[1][r] : -INFINITY;
-      const float l1 = has1 ? ctl->l_part[1][r] : 0.f;
-      const float m = fmaxf(m0, m1);
-      const float f0 = (m == -INFINITY) ? 0.f : ex2_approx(m0 - m);
-      const float f1 = (m == -INFINITY || !has1) ? 0.f : ex2_approx(m1 - m);
-      const float lt = l0 * f0 + l1 * f1;
-      const uint32_t tO0 = tmem + lane_base + kFwdTmemO + wg * 32;
-      uint32_t o0[32], o1[32];
-      __syncwarp();
-      tmem_ld32(tO0, o0);
-      if (has1) tmem_ld32(tO0 + kHeadDim, o1);
-      if (valid) {
-        const float inv_l = lt > 0.f ? 1.f / lt : 0.f;
-        const float g0 = f0 * inv_l, g1 = f1 * inv_l;
-        uint4* dst = reinterpret_cast<uint4*>(p.out + (static_cast<size_t>(t) * geo.Hq + h) * kHeadDim + wg * 32);
+    ok = warp_all(ok);
+    if constexpr (kTiles == 2) {
+      // ------------------------------------------ epilogue of tile wg alone
+      if (ok) {
+        tc_fence_after();
+        uint32_t o[kHeadDim];
+        __syncwarp();
+        tmem_ld64(tO, o);
+        if (valid) {
+          const float inv_l = l > 0.f ? 1.f / l : 0.f;
+          uint4* dst = reinterpret_cast<uint4*>(p.out + (static_cast<size_t>(t) * geo.Hq + h) * kHeadDim);
 #pragma unroll
-        for (int c8 = 0; c8 < 4; ++c8) {
-          float y[8];
-#pragma unroll
-          for (int u = 0; u < 8; ++u) {
-            const int c = 8 * c8 + u;
-            y[u] = __uint_as_float(o0[c]) * g0;
-            if (has1) y[u] = fmaf(__uint_as_float(o1[c]), g1, y[u]);
+          for (int c8 = 0; c8 < kHeadDim / 8; ++c8) {
+            uint4 v;
+            v.x = pack_bf16x2(__uint_as_float(o[8 * c8 + 0]) * inv_l, __uint_as_float(o[8 * c8 + 1]) * inv_l);
+            v.y = pack_bf16x2(__uint_as_float(o[8 * c8 + 2]) * inv_l, __uint_as_float(o[8 * c8 + 3]) * inv_l);
+            v.z = pack_bf16x2(__uint_as_float(o[8 * c8 + 4]) * inv_l, __uint_as_float(o[8 * c8 + 5]) * inv_l);
+            v.w = pack_bf16x2(__uint_as_float(o[8 * c8 + 6]) * inv_l, __uint_as_float(o[8 * c8 + 7]) * inv_l);
+            dst[c8] = v;
           }
-          uint4 v;
-          v.x = pack_bf16x2(y[0], y[1]);
-          v.y = pack_bf16x2(y[2], y[3]);
-          v.z = pack_bf16x2(y[4], y[5]);
-          v.w = pack_bf16x2(y[6], y[7]);
-          dst[c8] = v;
+          p.lse[static_cast<size_t>(h) * geo.T + t] = l > 0.f ? (m_ref + __log2f(l)) * kLn2 : -INFINITY;
         }
-        if (wg == 0) p.lse[static_cast<size_t>(h) * geo.T + t] = lt > 0.f ? (m + __log2f(lt)) * kLn2 : -INFINITY;
+      }
+    } else {
+      // ------------------------------------------------ merge and epilogue
+      // Each warpgroup publishes its (m, l); then warpgroup b writes output
+      // columns [32 b, 32 b + 32) of its rows from both accumulators.
+      ctl->m_part[wg][r] = m_ref;
+      ctl->l_part[wg][r] = l;
+      uint32_t merge_phase = 0;
+      mbar_arrive(&ctl->merge);
+      if (ok) ok = mbar_wait(&ctl->merge, merge_phase, abort, &g_device_error, kDevErrTimeoutEpilogue);
+      ok = warp_all(ok);
+      if (ok) {
+        tc_fence_after();
+        const bool has1 = w.n_half >= 2;  // warpgroup 1 saw at least one step
+        const float m0 = ctl->m_part[0][r], l0 = ctl->l_part[0][r];
+        const float m1 = has1 ? ctl->m_part[1][r] : -INFINITY;
+        const float l1 = has1 ? ctl->l_part[1][r] : 0.f;
+        const float m = fmaxf(m0, m1);
+        const float f0 = (m == -INFINITY) ? 0.f : ex2_approx(m0 - m);
+        const float f1 = (m == -INFINITY || !has1) ? 0.f : ex2_approx(m1 - m);
+        const float lt = l0 * f0 + l1 * f1;
+        const uint32_t tO0 = tmem + lane_base + kFwdTmemO + wg * 32;
+        uint32_t o0[32], o1[32];
+        __syncwarp();
+        tmem_ld32(tO0, o0);
+        if (has1) tmem_ld32(tO0 + kHeadDim, o1);
+        if (valid) {
+          const float inv_l = lt > 0.f ? 1.f / lt : 0.f;
+          const float g0 = f0 * inv_l, g1 = f1 * inv_l;
+          uint4* dst = reinterpret_cast<uint4*>(p.out + (static_cast<size_t>(t) * geo.Hq + h) * kHeadDim + wg * 32);
+  #pragma unroll
+          for (int c8 = 0; c8 < 4; ++c8) {
+            float y[8];
+  #pragma unroll
+            for (int u = 0; u < 8; ++u) {
+              const int c = 8 * c8 + u;
+              y[u] = __uint_as_float(o0[c]) * g0;
+              if (has1) y[u] = fmaf(__uint_as_float(o1[c]), g1, y[u]);
+            }
+            uint4 v;
+            v.x = pack_bf16x2(y[0], y[1]);
+            v.y = pack_bf16x2(y[2], y[3]);
+            v.z = pack_bf16x2(y[4], y[5]);
+            v.w = pack_bf16x2(y[6], y[7]);
+            dst[c8] = v;
+          }
+          if (wg == 0) p.lse[static_cast<size_t>(h) * geo.T + t] = lt > 0.f ? (m + __log2f(lt)) * kLn2 : -INFINITY;
+        }
       }
     }
   }

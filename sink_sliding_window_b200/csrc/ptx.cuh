@@ -112,6 +112,11 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   return mbar_wait_for(bar, parity, abort, err, code, kWaitLimitNs);
 }
 
+// A wait outcome made the same for every lane of the warp (false if any lane
+// gave up), so that a warp which gave up leaves its loop as one, before any
+// __syncwarp or .sync.aligned TMEM instruction that needs all its lanes.
+__device__ __forceinline__ bool warp_all(bool ok) { return __all_sync(0xffffffffu, ok); }
+
 // ----------------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");

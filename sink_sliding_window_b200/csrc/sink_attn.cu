@@ -15,6 +15,7 @@
 #include "common.cuh"
 #include "tma_host.cuh"
 #include "fwd_kernel.cuh"
+#include "fwd_pair_kernel.cuh"
 #include "bwd_kernels.cuh"
 #include "decode_kernel.cuh"
 
@@ -62,6 +63,52 @@ sink_attn_status check_dims(const sink_attn_dims* d, const int* cu_seqlens, bool
   geo->window = window > 0 ? window : 0;
   if (!packed && d->total_tokens > 0 && d->max_seqlen <= 0) return SINK_ATTN_ERR_SHAPE;
   return SINK_ATTN_OK;
+}
+
+// Checks of a forward call (both forward entry points): sizes, then (for
+// T > 0) pointers and alignment.  Fills the geometry.
+sink_attn_status check_fwd_args(const sink_attn_dims* d, const void* q, const void* k, const void* v,
+                                const float* sinks, const int* cu_seqlens, int window, float scale, const void* out,
+                                const float* lse, Geometry* geo) {
+  sink_attn_status st = check_dims(d, cu_seqlens, cu_seqlens != nullptr, window, scale, geo);
+  if (st != SINK_ATTN_OK || geo->T == 0) return st;
+  if (!q || !k || !v || !sinks || !out || !lse) return SINK_ATTN_ERR_NULL;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) ||
+      (reinterpret_cast<uintptr_t>(lse) & 3u) || (reinterpret_cast<uintptr_t>(sinks) & 3u) ||
+      (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u))
+    return SINK_ATTN_ERR_ALIGN;
+  return SINK_ATTN_OK;
+}
+
+// Largest window for which sink_attn_fwd takes the two-tile kernel.
+constexpr int kFwdTwoTileMaxWindow = 0;
+
+// The forward kernel sink_attn_fwd runs for these sizes.  Sliding-window
+// layers whose query tiles see only a few 64-key steps take two tiles per CTA
+// (set-up and epilogue are paid once per two tiles, and one K/V stream serves
+// both); longer key ranges take one tile per CTA, whose two warpgroups split
+// the tile's steps.
+int fwd_auto_kernel(const Geometry& geo) {
+  if (geo.window > 0 && geo.window <= kFwdTwoTileMaxWindow) return SINK_ATTN_FWD_TWO_TILES;
+  return SINK_ATTN_FWD_ONE_TILE;
+}
+
+// 3-D bf16 view [outer][mid][inner] with a box {box_inner, 1, box_outer}
+// under the given swizzle: the pair forward's half-steps of K (32 keys x 64
+// dims, 128-byte rows) and V (64 keys x 32 dims, 64-byte rows).
+bool make_map_3d_box(CUtensorMap* map, const void* base, int inner, int mid, int outer, int box_inner,
+                     int box_outer, CUtensorMapSwizzle swizzle) {
+  EncodeTiledFn enc = get_encode_tiled();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(mid),
+                        static_cast<cuuint64_t>(outer)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(inner) * 2, static_cast<cuuint64_t>(inner) * mid * 2};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(box_inner), 1, static_cast<cuuint32_t>(box_outer)};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
 }
 
 // Events registered by sink_attn_profile_events: [which][begin/end].
@@ -228,25 +275,45 @@ int sink_attn_fwd_launches(const sink_attn_dims* d) {
 sink_attn_status sink_attn_fwd(const sink_attn_dims* d, const void* q, const void* k, const void* v,
                                const float* sinks, const int* cu_seqlens, int window, float scale, void* out,
                                float* lse, void* stream) {
+  return sink_attn_fwd_with(d, q, k, v, sinks, cu_seqlens, window, scale, out, lse, SINK_ATTN_FWD_AUTO, stream);
+}
+
+sink_attn_status sink_attn_fwd_pair(const sink_attn_dims* d, const void* q, const void* k, const void* v,
+                                    const float* sinks, const int* cu_seqlens, int window, float scale, void* out,
+                                    float* lse, void* stream) {
+  return sink_attn_fwd_with(d, q, k, v, sinks, cu_seqlens, window, scale, out, lse, SINK_ATTN_FWD_CTA_PAIR,
+                            stream);
+}
+
+int sink_attn_fwd_kernel_for(const sink_attn_dims* d, int window) {
   Geometry geo;
-  sink_attn_status st = check_dims(d, cu_seqlens, cu_seqlens != nullptr, window, scale, &geo);
-  if (st != SINK_ATTN_OK) return st;
-  if (geo.T == 0) return SINK_ATTN_OK;
-  if (!q || !k || !v || !sinks || !out || !lse) return SINK_ATTN_ERR_NULL;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) ||
-      (reinterpret_cast<uintptr_t>(lse) & 3u) || (reinterpret_cast<uintptr_t>(sinks) & 3u) ||
-      (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u))
-    return SINK_ATTN_ERR_ALIGN;
+  if (check_dims(d, nullptr, true, window, 1.f, &geo) != SINK_ATTN_OK) return -1;
+  return fwd_auto_kernel(geo);
+}
+
+sink_attn_status sink_attn_fwd_with(const sink_attn_dims* d, const void* q, const void* k, const void* v,
+                                    const float* sinks, const int* cu_seqlens, int window, float scale, void* out,
+                                    float* lse, int kernel, void* stream) {
+  if (kernel < SINK_ATTN_FWD_AUTO || kernel > SINK_ATTN_FWD_CTA_PAIR) return SINK_ATTN_ERR_UNSUPPORTED;
+  Geometry geo;
+  sink_attn_status st = check_fwd_args(d, q, k, v, sinks, cu_seqlens, window, scale, out, lse, &geo);
+  if (st != SINK_ATTN_OK || geo.T == 0) return st;
+  if (kernel == SINK_ATTN_FWD_AUTO) kernel = fwd_auto_kernel(geo);
 
   const int G = 1 << geo.G_log2;
+  const bool pair = kernel == SINK_ATTN_FWD_CTA_PAIR;
   CUtensorMap tq, tk, tv;
-  if (!make_map_3d(&tq, q, kHeadDim, geo.Hq, geo.T, G, 1 << geo.P_log2) ||
-      !make_map_3d(&tk, k, kHeadDim, geo.Hkv, geo.T, 1, kBlockN) ||
-      !make_map_3d(&tv, v, kHeadDim, geo.Hkv, geo.T, 1, kBlockN))
+  if (!make_map_3d(&tq, q, kHeadDim, geo.Hq, geo.T, G, 1 << geo.P_log2)) return SINK_ATTN_ERR_CUDA;
+  if (pair) {
+    // Each CTA of a pair loads 32 keys x 64 dims of K and 64 keys x 32 dims
+    // of V per 64-key step.
+    if (!make_map_3d_box(&tk, k, kHeadDim, geo.Hkv, geo.T, kHeadDim, kHalfN / 2, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map_3d_box(&tv, v, kHeadDim, geo.Hkv, geo.T, kHeadDim / 2, kHalfN, CU_TENSOR_MAP_SWIZZLE_64B))
+      return SINK_ATTN_ERR_CUDA;
+  } else if (!make_map_3d(&tk, k, kHeadDim, geo.Hkv, geo.T, 1, kBlockN) ||
+             !make_map_3d(&tv, v, kHeadDim, geo.Hkv, geo.T, 1, kBlockN)) {
     return SINK_ATTN_ERR_CUDA;
-
-  static SmemAttrOnce smem_set;
-  if (!smem_set.ensure(sink_attn_fwd_kernel, kFwdSmemBytes)) return SINK_ATTN_ERR_CUDA;
+  }
 
   FwdParams p;
   p.geo = geo;
@@ -254,13 +321,46 @@ sink_attn_status sink_attn_fwd(const sink_attn_dims* d, const void* q, const voi
   p.sinks = sinks;
   p.out = static_cast<__nv_bfloat16*>(out);
   p.lse = lse;
-  const int64_t grid = static_cast<int64_t>(geo.num_qblocks) * geo.Hkv;
+  // One tile: a CTA per (query tile, head g); two tiles and pairs: a CTA per
+  // two query tiles, or a pair of CTAs per two query tiles.
+  const int64_t units = kernel == SINK_ATTN_FWD_ONE_TILE ? geo.num_qblocks : (geo.num_qblocks + 1) / 2;
+  const int64_t grid = units * geo.Hkv * (pair ? 2 : 1);
   if (grid > 0x7fffffff) return SINK_ATTN_ERR_UNSUPPORTED;
   cudaStream_t st_ = static_cast<cudaStream_t>(stream);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
+  cfg.blockDim = dim3(kFwdThreads, 1, 1);
+  cfg.stream = st_;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cudaError_t e;
   if (g_profile_events[0][0]) cudaEventRecord(g_profile_events[0][0], st_);
-  sink_attn_fwd_kernel<<<static_cast<unsigned>(grid), kFwdThreads, kFwdSmemBytes, st_>>>(tq, tk, tv, p);
+  if (kernel == SINK_ATTN_FWD_ONE_TILE) {
+    static SmemAttrOnce smem_set;
+    cfg.dynamicSmemBytes = fwd_smem_bytes<1>();
+    e = smem_set.ensure(sink_attn_fwd_kernel<1>, cfg.dynamicSmemBytes)
+            ? cudaLaunchKernelEx(&cfg, sink_attn_fwd_kernel<1>, tq, tk, tv, p)
+            : cudaErrorInvalidValue;
+  } else if (kernel == SINK_ATTN_FWD_TWO_TILES) {
+    static SmemAttrOnce smem_set;
+    cfg.dynamicSmemBytes = fwd_smem_bytes<2>();
+    e = smem_set.ensure(sink_attn_fwd_kernel<2>, cfg.dynamicSmemBytes)
+            ? cudaLaunchKernelEx(&cfg, sink_attn_fwd_kernel<2>, tq, tk, tv, p)
+            : cudaErrorInvalidValue;
+  } else {
+    static SmemAttrOnce smem_set;
+    cfg.dynamicSmemBytes = kF2SmemBytes;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = smem_set.ensure(sink_attn_fwd_pair_kernel, cfg.dynamicSmemBytes)
+            ? cudaLaunchKernelEx(&cfg, sink_attn_fwd_pair_kernel, tq, tk, tv, p)
+            : cudaErrorInvalidValue;
+  }
   if (g_profile_events[0][1]) cudaEventRecord(g_profile_events[0][1], st_);
-  return cudaPeekAtLastError() == cudaSuccess ? SINK_ATTN_OK : SINK_ATTN_ERR_CUDA;
+  return e == cudaSuccess ? SINK_ATTN_OK : SINK_ATTN_ERR_CUDA;
 }
 
 size_t sink_attn_bwd_workspace_size(const sink_attn_dims* d) {

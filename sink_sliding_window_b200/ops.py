@@ -25,7 +25,7 @@ STATUS = {
     7: "SINK_ATTN_ERR_WORKSPACE",
 }
 
-EXPORTS = ("sink_attn_fwd", "sink_attn_bwd", "sink_attn_bwd_workspace_size", "sink_attn_status_string",
+EXPORTS = ("sink_attn_fwd", "sink_attn_fwd_pair", "sink_attn_fwd_with", "sink_attn_fwd_kernel_for", "sink_attn_bwd", "sink_attn_bwd_workspace_size", "sink_attn_status_string",
            "sink_attn_last_device_error", "sink_attn_device_error", "sink_attn_fwd_launches", "sink_attn_bwd_launches", "sink_attn_profile_events",
            "sink_attn_decode", "sink_attn_decode_workspace_size", "sink_attn_decode_launches",
            "sink_attn_decode_e4m3", "sink_attn_decode_e4m3_f8pv", "sink_attn_selftest_wait")
@@ -65,6 +65,12 @@ def load():
         DP = ctypes.POINTER(Dims)
         L.sink_attn_fwd.argtypes = [DP, P, P, P, P, P, I, ctypes.c_float, P, P, P]
         L.sink_attn_fwd.restype = I
+        L.sink_attn_fwd_pair.argtypes = L.sink_attn_fwd.argtypes
+        L.sink_attn_fwd_pair.restype = I
+        L.sink_attn_fwd_with.argtypes = [DP, P, P, P, P, P, I, ctypes.c_float, P, P, I, P]
+        L.sink_attn_fwd_with.restype = I
+        L.sink_attn_fwd_kernel_for.argtypes = [DP, I]
+        L.sink_attn_fwd_kernel_for.restype = I
         L.sink_attn_bwd.argtypes = [DP, P, P, P, P, P, I, ctypes.c_float, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]
         L.sink_attn_bwd.restype = I
         L.sink_attn_bwd_workspace_size.argtypes = [DP]
@@ -141,11 +147,16 @@ def _geometry(q, k, cu_seqlens, batch, max_seqlen):
     return make_dims(T, Hq, Hkv, D, batch, max_seqlen), T, Hq, Hkv, D
 
 
+# sink_attn_fwd_kernel_id values of the C ABI.
+FWD_KERNELS = {"auto": 0, "one_tile": 1, "two_tiles": 2, "pair": 3}
+
+
 def fwd(q, k, v, sinks, cu_seqlens=None, window=0, scale=None, *, batch=None, max_seqlen=None, out=None, lse=None,
-        stream=None):
-    """sink_attn_fwd.  q [T,Hq,D] (or [B,S,Hq,D]), k/v [T,Hkv,D] bf16 CUDA;
-    sinks [Hq] fp32; cu_seqlens int32 [B+1] CUDA or None.
-    Returns (out like q, lse [Hq, T] fp32)."""
+        stream=None, kernel="auto"):
+    """sink_attn_fwd (kernel="auto"), or sink_attn_fwd_with one of the
+    library's forward kernels ("one_tile", "two_tiles", "pair").  q [T,Hq,D]
+    (or [B,S,Hq,D]), k/v [T,Hkv,D] bf16 CUDA; sinks [Hq] fp32; cu_seqlens
+    int32 [B+1] CUDA or None.  Returns (out like q, lse [Hq, T] fp32)."""
     dims, T, Hq, Hkv, D = _geometry(q, k, cu_seqlens, batch, max_seqlen)
     if scale is None:
         scale = D ** -0.5
@@ -153,11 +164,37 @@ def fwd(q, k, v, sinks, cu_seqlens=None, window=0, scale=None, *, batch=None, ma
         out = torch.empty_like(q)
     if lse is None:
         lse = torch.empty((Hq, T), dtype=torch.float32, device=q.device)
-    st = load().sink_attn_fwd(ctypes.byref(dims), _ptr(q), _ptr(k), _ptr(v), _ptr(sinks), _ptr(cu_seqlens),
-                              int(window), float(scale), _ptr(out), _ptr(lse), _stream_handle(stream))
+    args = (ctypes.byref(dims), _ptr(q), _ptr(k), _ptr(v), _ptr(sinks), _ptr(cu_seqlens), int(window), float(scale),
+            _ptr(out), _ptr(lse))
+    if kernel == "auto":
+        name, st = "sink_attn_fwd", load().sink_attn_fwd(*args, _stream_handle(stream))
+    else:
+        name, st = "sink_attn_fwd_with", load().sink_attn_fwd_with(*args, FWD_KERNELS[kernel], _stream_handle(stream))
     if st != 0:
-        raise SinkAttnError(st, "sink_attn_fwd")
+        raise SinkAttnError(st, name)
     return out, lse
+
+
+def fwd_pair(q, k, v, sinks, cu_seqlens=None, window=0, scale=None, **kw):
+    """sink_attn_fwd_pair: the forward on CTA pairs (tcgen05 M = 256)."""
+    dims, T, Hq, Hkv, D = _geometry(q, k, cu_seqlens, kw.get("batch"), kw.get("max_seqlen"))
+    out = kw.get("out")
+    lse = kw.get("lse")
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty((Hq, T), dtype=torch.float32, device=q.device) if lse is None else lse
+    st = load().sink_attn_fwd_pair(ctypes.byref(dims), _ptr(q), _ptr(k), _ptr(v), _ptr(sinks), _ptr(cu_seqlens),
+                                   int(window), float(D ** -0.5 if scale is None else scale), _ptr(out), _ptr(lse),
+                                   _stream_handle(kw.get("stream")))
+    if st != 0:
+        raise SinkAttnError(st, "sink_attn_fwd_pair")
+    return out, lse
+
+
+def fwd_kernel_for(T, Hq, Hkv, D, batch, max_seqlen, window) -> str:
+    """Name of the forward kernel sink_attn_fwd runs for these sizes."""
+    d = make_dims(T, Hq, Hkv, D, batch, max_seqlen)
+    k = int(load().sink_attn_fwd_kernel_for(ctypes.byref(d), int(window)))
+    return {v: n for n, v in FWD_KERNELS.items()}.get(k, "invalid")
 
 
 def bwd_workspace_size(T, Hq, Hkv, D, batch, max_seqlen) -> int:

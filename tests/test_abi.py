@@ -48,8 +48,12 @@ def dims(**kw):
 FAKE = ctypes.c_void_p(1 << 20)  # 16-byte aligned, never dereferenced: validation fails first
 
 
-def call_fwd(L, d, q=FAKE, k=FAKE, v=FAKE, sinks=FAKE, cu=None, window=0, scale=0.125, out=FAKE, lse=FAKE):
-    return L.sink_attn_fwd(ctypes.byref(d), q, k, v, sinks, cu, window, scale, out, lse, None)
+FWD_ENTRIES = ("sink_attn_fwd", "sink_attn_fwd_pair")
+
+
+def call_fwd(L, d, q=FAKE, k=FAKE, v=FAKE, sinks=FAKE, cu=None, window=0, scale=0.125, out=FAKE, lse=FAKE,
+             entry="sink_attn_fwd"):
+    return getattr(L, entry)(ctypes.byref(d), q, k, v, sinks, cu, window, scale, out, lse, None)
 
 
 @pytest.mark.parametrize("bad,code", [
@@ -61,26 +65,50 @@ def call_fwd(L, d, q=FAKE, k=FAKE, v=FAKE, sinks=FAKE, cu=None, window=0, scale=
     (dict(Hkv=0), 2),
     (dict(batch=0, max_seqlen=0), 2),
 ])
-def test_fwd_rejects_bad_shapes(L, bad, code):
-    assert call_fwd(L, dims(**bad)) == code
+@pytest.mark.parametrize("entry", FWD_ENTRIES)
+def test_fwd_rejects_bad_shapes(L, bad, code, entry):
+    assert call_fwd(L, dims(**bad), entry=entry) == code
 
 
-def test_fwd_rejects_null_and_misaligned(L):
-    assert L.sink_attn_fwd(None, FAKE, FAKE, FAKE, FAKE, None, 0, 0.125, FAKE, FAKE, None) == 1
-    assert call_fwd(L, dims(), q=None) == 1
-    assert call_fwd(L, dims(), lse=None) == 1
-    assert call_fwd(L, dims(), k=ctypes.c_void_p((1 << 20) + 8)) == 3
-    assert call_fwd(L, dims(), out=ctypes.c_void_p((1 << 20) + 2)) == 3
+@pytest.mark.parametrize("entry", FWD_ENTRIES)
+def test_fwd_rejects_null_and_misaligned(L, entry):
+    assert getattr(L, entry)(None, FAKE, FAKE, FAKE, FAKE, None, 0, 0.125, FAKE, FAKE, None) == 1
+    assert call_fwd(L, dims(), q=None, entry=entry) == 1
+    assert call_fwd(L, dims(), lse=None, entry=entry) == 1
+    assert call_fwd(L, dims(), k=ctypes.c_void_p((1 << 20) + 8), entry=entry) == 3
+    assert call_fwd(L, dims(), out=ctypes.c_void_p((1 << 20) + 2), entry=entry) == 3
 
 
-def test_fwd_rejects_bad_scale(L):
+@pytest.mark.parametrize("entry", FWD_ENTRIES)
+def test_fwd_rejects_bad_scale(L, entry):
     for s in (0.0, -0.125, float("inf"), float("nan")):
-        assert call_fwd(L, dims(), scale=s) == 4
+        assert call_fwd(L, dims(), scale=s, entry=entry) == 4
 
 
-def test_fwd_empty_is_noop(L):
+@pytest.mark.parametrize("entry", FWD_ENTRIES)
+def test_fwd_empty_is_noop(L, entry):
     # T = 0: valid, nothing to do, no pointer is touched.
-    assert call_fwd(L, dims(T=0, batch=0, max_seqlen=0), q=None, k=None, v=None, out=None, lse=None) == 0
+    assert call_fwd(L, dims(T=0, batch=0, max_seqlen=0), q=None, k=None, v=None, out=None, lse=None,
+                    entry=entry) == 0
+
+
+def test_fwd_with_rejects_unknown_kernel(L):
+    # kernel ids other than SINK_ATTN_FWD_AUTO .. SINK_ATTN_FWD_CTA_PAIR: SINK_ATTN_ERR_UNSUPPORTED
+    for kid in (-1, 4, 99):
+        assert L.sink_attn_fwd_with(ctypes.byref(dims()), FAKE, FAKE, FAKE, FAKE, None, 0, 0.125, FAKE, FAKE, kid,
+                                    None) == 4
+    # and the same validation as sink_attn_fwd for a known id
+    assert L.sink_attn_fwd_with(ctypes.byref(dims(D=128)), FAKE, FAKE, FAKE, FAKE, None, 0, 0.125, FAKE, FAKE, 2,
+                                None) == 4
+    assert L.sink_attn_fwd_with(ctypes.byref(dims()), None, FAKE, FAKE, FAKE, None, 0, 0.125, FAKE, FAKE, 3,
+                                None) == 1
+
+
+def test_fwd_kernel_for(L):
+    for window in (0, 1, 128, 4096):
+        assert L.sink_attn_fwd_kernel_for(ctypes.byref(dims()), window) in (1, 2, 3)
+    assert L.sink_attn_fwd_kernel_for(ctypes.byref(dims(D=32)), 0) == -1
+    assert ops.fwd_kernel_for(256, 8, 2, 64, 2, 128, 0) in ("one_tile", "two_tiles", "pair")
 
 
 def test_bwd_workspace_and_validation(L):

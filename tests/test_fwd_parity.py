@@ -1,4 +1,5 @@
-"""sink_attn_fwd (CUDA, through the C ABI) against the fp64 oracle on the
+"""The forward kernels (CUDA, through the C ABI: sink_attn_fwd_with with each
+kernel, sink_attn_fwd, sink_attn_fwd_pair) against the fp64 oracle on the
 same seeded bf16 inputs: whole tensors on small cases that still span several
 tiles and a ragged tail, sampled rows (every head) at the full workload
 sizes, and the edge cases of the method (tiny and single-token documents,
@@ -13,13 +14,30 @@ from tests.gpu_util import TOL_LSE, TOL_OUT, check, dev, dev_bf16, host_f64, run
 pytestmark = pytest.mark.gpu
 
 
-@pytest.fixture(scope="module")
-def ops():
+class _KernelOps:
+    """The binding with fwd pinned to one of the library's forward kernels
+    (through sink_attn_fwd_with)."""
+
+    def __init__(self, mod, kernel):
+        self._mod = mod
+        self.kernel = kernel
+
+    def fwd(self, *args, **kw):
+        return self._mod.fwd(*args, kernel=self.kernel, **kw)
+
+    def __getattr__(self, name):
+        return getattr(self._mod, name)
+
+
+@pytest.fixture(scope="module", params=["one_tile", "two_tiles", "pair"])
+def ops(request):
+    """Every case runs through each forward kernel: one query tile per CTA,
+    two tiles per CTA, and CTA pairs (M = 256)."""
     import torch
     from sink_sliding_window_b200 import build, ops as _ops
     assert torch.cuda.is_available()
     build.build()
-    return _ops
+    return _KernelOps(_ops, request.param)
 
 
 @pytest.mark.parametrize("name", ["tiny:w32", "tiny:full"])
@@ -150,3 +168,39 @@ def test_deterministic(ops):
     o1, l1 = run_fwd(w, a, ops)
     o2, l2 = run_fwd(w, a, ops)
     assert (o1 == o2).all() and (l1 == l2).all()
+
+
+@pytest.fixture(scope="module")
+def ops_mod():
+    import torch
+    from sink_sliding_window_b200 import build, ops as _ops
+    assert torch.cuda.is_available()
+    build.build()
+    return _ops
+
+
+@pytest.mark.parametrize("name", ["prefill4k:full", "prefill4k:w128"])
+def test_kernels_agree(ops_mod, name):
+    """sink_attn_fwd, sink_attn_fwd_pair and every kernel of
+    sink_attn_fwd_with agree to rounding on the prefill shapes (each is also
+    checked against the oracle above), and sink_attn_fwd is bit-identical to
+    the kernel it reports through sink_attn_fwd_kernel_for."""
+    import torch
+    w = synth.workload(name)
+    a = w.generate()
+    o_auto, l_auto = run_fwd(w, a, ops_mod)
+    chosen = ops_mod.fwd_kernel_for(w.T, w.Hq, w.Hkv, w.D, w.batch, w.max_seqlen, w.window)
+    assert chosen in ("one_tile", "two_tiles", "pair")
+    scale_o = float(o_auto.float().abs().max())
+    for kn in ("one_tile", "two_tiles", "pair"):
+        o, l = run_fwd(w, a, _KernelOps(ops_mod, kn))
+        if kn == chosen:
+            assert (o == o_auto).all() and (l == l_auto).all()
+        assert float((o.float() - o_auto.float()).abs().max()) <= 1e-2 * scale_o
+        assert float((l - l_auto).abs().max()) <= 1e-3 * float(l_auto.abs().max())
+        assert torch.isfinite(l).all()
+    o_p, l_p = ops_mod.fwd_pair(dev_bf16(a["q"]), dev_bf16(a["k"]), dev_bf16(a["v"]), dev(a["sinks"]), None,
+                                w.window, w.scale, batch=w.batch, max_seqlen=w.uniform_seqlen)
+    o_w, l_w = run_fwd(w, a, _KernelOps(ops_mod, "pair"))
+    torch.cuda.synchronize()
+    assert (o_p == o_w).all() and (l_p == l_w).all()
