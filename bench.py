@@ -320,7 +320,7 @@ def measure_layers(torch, ops, stream, q, k, v, sinks, dout, outs, grads, ws, it
                 entry.setdefault("fwd_kernels", {})[name.split(":")[1]] = r
             else:
                 entry[name] = r
-        entry["fwd"]["kernel"] = ops.fwd_kernel_for(T, HQ, HKV, D, B, S, W)
+        entry["fwd"]["kernel"] = ops.fwd_kernel_for(B * S, HQ, HKV, D, B, S, W)
         entry["peak_GBps"] = hbm
         entry["peak_source"] = f"{kind} hbm_gbs"
         res.append(entry)

@@ -86,7 +86,8 @@ typedef struct {
 /* Forward.  q [T][Hq][D] bf16, k, v [T][Hkv][D] bf16, sinks [Hq] fp32 (may
  * hold -INFINITY), cu_seqlens int32 [batch+1] on the device or NULL (then
  * every document has length max_seqlen).  Writes out [T][Hq][D] bf16 and
- * lse [Hq][T] fp32 (natural log, sink included).  T = 0 is a no-op. */
+ * lse [Hq][T] fp32 (natural log, sink included).  T = 0 is a no-op.  Runs
+ * the kernel sink_attn_fwd_kernel_for() names (two query tiles per CTA). */
 sink_attn_status sink_attn_fwd(const sink_attn_dims* dims,
                                const void* q, const void* k, const void* v,
                                const float* sinks, const int* cu_seqlens,

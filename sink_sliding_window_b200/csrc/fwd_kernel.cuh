@@ -1,9 +1,9 @@
 // Forward kernel: causal GQA attention with a per-head sink logit, sliding
 // window and packed documents, on sm_100a tensor cores.
 //
-// Work unit: one CTA owns one query tile = (128 / G) consecutive tokens x the
-// G query heads of one key/value head g, i.e. 128 MMA rows, row r <->
-// (token t0 + r / G, head g*G + r % G).  Because q is [T][Hq][D], the G heads
+// Query tile: (128 / G) consecutive tokens x the G query heads of one
+// key/value head g, i.e. 128 MMA rows, row r <-> (token t0 + r / G, head
+// g*G + r % G).  In the one-tile mode (kTiles = 1) a CTA owns one tile.  Because q is [T][Hq][D], the G heads
 // of a group are contiguous and a single 3-D TMA box {64, G, 128/G} lands the
 // tile in exactly this row order.  Every key/value tile that is loaded serves
 // all G heads of the group.
@@ -31,15 +31,16 @@
 // Tiles outside the causal / window / document range are never visited; only
 // the edge steps apply an element mask.
 //
-// Two-tile mode (kTiles = 2, for short key ranges such as sliding-window
-// layers, where a one-tile CTA does only a few steps between its set-up and
-// its epilogue): the CTA owns two adjacent query tiles of the same head g,
-// warpgroup b takes every step of tile b (its own S/P buffer, O_b, running
-// max and sum, no merge), and one K/V stream over the union of the two
-// tiles' key ranges serves both; each warpgroup masks its own rows.  The MMA
-// issuer serves the warpgroups in turn (PV_b and S_b of the next step as soon
-// as P_b is written), so one warpgroup's exponentials overlap the other's
-// S round trip, as the alternating steps do in the one-tile mode.
+// Two-tile mode (kTiles = 2, what sink_attn_fwd runs): the CTA owns two
+// adjacent query tiles of the same head g, warpgroup b takes every step of
+// tile b (its own S/P buffer, O_b, running max and sum, no merge), and one
+// K/V stream over the union of the two tiles' key ranges serves both; each
+// warpgroup masks its own rows.  The MMA issuer serves the warpgroups in turn
+// (PV_b and S_b of the next step as soon as P_b is written), so one
+// warpgroup's exponentials overlap the other's S round trip, as the
+// alternating steps do in the one-tile mode.  Set-up, first loads and
+// epilogue are paid once per two tiles, which matters most on sliding-window
+// layers (a tile sees only 3-4 key steps there).
 //
 // Warp roles (320 threads, 2 CTAs per SM): warps 0-7 softmax + epilogue (two
 // warpgroups), warp 8 TMA producer, warp 9 TMEM allocator + MMA issuer.
