@@ -23,6 +23,7 @@ import argparse
 import hashlib
 import json
 import os
+import statistics
 import subprocess
 import sys
 import time
@@ -276,13 +277,38 @@ def measure_decode(torch, ops, stream, iters=20):
     return res
 
 
-def measure_layers(torch, ops, stream, q, k, v, sinks, dout, outs, grads, ws, iters=20):
-    """Forward and backward of each layer alone (CUDA events on the launching
-    stream, mean over `iters` calls after 3 warm-up calls): TFLOP/s on the
+def time_calls(torch, stream, fns, iters, rounds=4, warm=2):
+    """ms per call of each function in `fns`: CUDA events on the launching
+    stream around `iters` calls, in `rounds` rounds that take the functions in
+    turn (in reverse order every other round), so that clock changes under the
+    power cap fall on all of them alike; the median over the rounds."""
+    for fn in fns.values():
+        for _ in range(warm):
+            fn()
+    torch.cuda.synchronize()
+    keys = list(fns)
+    times = {k: [] for k in keys}
+    for r in range(rounds):
+        for k in (keys if r % 2 == 0 else keys[::-1]):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(iters):
+                fns[k]()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            times[k].append(e0.elapsed_time(e1) / iters)
+    return {k: statistics.median(v) for k, v in times.items()}
+
+
+def measure_layers(torch, ops, stream, q, k, v, sinks, dout, outs, grads, ws, iters=10):
+    """Forward and backward of each layer alone (time_calls: CUDA events on
+    the launching stream, the forward kernels taken in turn): TFLOP/s on the
     counted pairs, and GB/s of the layer's minimum DRAM bytes (every input
     read once, every output written once) against the measured HBM peak; the
-    window-128 layers are judged on the latter.  q, dout, out and dq (134 MB
-    each) exceed the 126 MB L2, so no flush between calls."""
+    window-128 layers are judged on the latter.  "fwd" is sink_attn_fwd (the
+    kernel it picks is named), "fwd_kernels" each forward kernel through
+    sink_attn_fwd_with.  q, dout, out and dq (134 MB each) exceed the 126 MB
+    L2, so no flush between calls."""
     _, hbm, kind = read_peaks()
     nb = lambda *ts: sum(t.numel() * t.element_size() for t in ts)  # noqa: E731
     res = []
@@ -290,32 +316,25 @@ def measure_layers(torch, ops, stream, q, k, v, sinks, dout, outs, grads, ws, it
         o, l = outs[W]
         dq, dk, dv, ds = grads[W]
         kw = dict(batch=B, max_seqlen=S, stream=stream)
-        calls = {
-            "fwd": (lambda: ops.fwd(q, k, v, sinks, None, W, 0.125, out=o, lse=l, **kw),
-                    nb(q, k, v, sinks) + nb(o, l)),
-            "bwd": (lambda: ops.bwd(q, k, v, sinks, o, l, dout, None, W, 0.125, dq=dq, dk=dk, dv=dv, dsinks=ds,
-                                    workspace=ws, **kw),
-                    nb(q, k, v, sinks, o, l, dout) + nb(dq, dk, dv, ds)),
-        }
+        fwd_bytes = nb(q, k, v, sinks) + nb(o, l)
+        bwd_bytes = nb(q, k, v, sinks, o, l, dout) + nb(dq, dk, dv, ds)
+        fwd = {"fwd": lambda: ops.fwd(q, k, v, sinks, None, W, 0.125, out=o, lse=l, **kw)}
         for kn in FWD_KERNEL_NAMES:
-            calls["fwd:" + kn] = ((lambda kn=kn: ops.fwd(q, k, v, sinks, None, W, 0.125, out=o, lse=l, kernel=kn,
-                                                         **kw)),
-                                  calls["fwd"][1])
+            fwd["fwd:" + kn] = (lambda kn=kn: ops.fwd(q, k, v, sinks, None, W, 0.125, out=o, lse=l, kernel=kn,
+                                                      **kw))
+        ms = time_calls(torch, stream, fwd, iters)
+        # the backward reads the saved out / lse of the last forward call
+        ops.fwd(q, k, v, sinks, None, W, 0.125, out=o, lse=l, **kw)
+        ms.update(time_calls(torch, stream, {"bwd": lambda: ops.bwd(q, k, v, sinks, o, l, dout, None, W, 0.125, dq=dq,
+                                                                      dk=dk, dv=dv, dsinks=ds, workspace=ws, **kw)},
+                             iters, rounds=2))
         fl = dict(zip(("fwd", "bwd"), layer_flops(W)))
         entry = {"window": W, "workload": f"{WORKLOAD} ({'window %d' % W if W > 0 else 'full causal'})"}
-        for name, (fn, min_bytes) in calls.items():
-            for _ in range(3):
-                fn()
-            torch.cuda.synchronize()
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            for _ in range(iters):
-                fn()
-            e1.record(stream)
-            torch.cuda.synchronize()
-            ms = e0.elapsed_time(e1) / iters
-            r = {"ms": ms, "tflops": fl[name.split(":")[0]] / ms / 1e9, "min_bytes": min_bytes,
-                 "GBps": min_bytes / ms / 1e6, "hbm_frac": min_bytes / ms / 1e6 / hbm}
+        for name, t in ms.items():
+            base = name.split(":")[0]
+            mb = fwd_bytes if base == "fwd" else bwd_bytes
+            r = {"ms": t, "tflops": fl[base] / t / 1e9, "min_bytes": mb, "GBps": mb / t / 1e6,
+                 "hbm_frac": mb / t / 1e6 / hbm}
             if ":" in name:
                 entry.setdefault("fwd_kernels", {})[name.split(":")[1]] = r
             else:
@@ -374,11 +393,11 @@ def layer_buffers(torch, ops, w, t):
 def measure_extra(torch, ops, stream, iters=5):
     """Forward and backward of the long-context (one 61,440-token document,
     sinks ~N(0, 2^2)) and packed-document (65,536 tokens in documents of
-    ~U[256, 8192] tokens) workloads, window 128 and full causal, each call
-    timed alone with CUDA events on the launching stream (mean of `iters`
-    after 2 warm-up calls; every input exceeds the L2, so no flush).  Full
-    causal: TFLOP/s on the counted pairs and % of the measured bf16 peak;
-    window 128: GB/s of the layer's minimum bytes against the HBM peak."""
+    ~U[256, 8192] tokens) workloads, window 128 and full causal, timed with
+    time_calls (CUDA events on the launching stream, the forward kernels in
+    turn; every input exceeds the L2, so no flush).  Full causal: TFLOP/s on
+    the counted pairs and % of the measured bf16 peak; window 128: GB/s of
+    the layer's minimum bytes against the HBM peak."""
     peak, hbm, kind = read_peaks()
     nb = lambda *ts: sum(x.numel() * x.element_size() for x in ts if x is not None)  # noqa: E731
     res = {}
@@ -395,22 +414,20 @@ def measure_extra(torch, ops, stream, iters=5):
             p = pairs(w.cu_seqlens, window, w.Hq)
             lay = {"window": window}
             fwd_mb = nb(t["q"], t["k"], t["v"], t["sinks"], o, l)
-            cases = [("fwd", f, 4 * D * p, fwd_mb)]
-            cases += [("fwd:" + kn, (lambda kn=kn: f(kn)), 4 * D * p, fwd_mb) for kn in FWD_KERNEL_NAMES]
-            cases += [("bwd", b, 10 * D * p, nb(t["q"], t["k"], t["v"], t["sinks"], o, l, t["dout"], dq, dk, dv, ds))]
-            for name, fn, flops, mb in cases:
-                for _ in range(2):
-                    fn()
-                torch.cuda.synchronize()
-                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                e0.record(stream)
-                for _ in range(iters):
-                    fn()
-                e1.record(stream)
-                torch.cuda.synchronize()
-                ms = e0.elapsed_time(e1) / iters
-                r = {"ms": ms, "tflops": flops / ms / 1e9, "pct_of_peak": 100.0 * flops / ms / 1e9 / peak,
-                     "min_bytes": mb, "GBps": mb / ms / 1e6, "hbm_frac": mb / ms / 1e6 / hbm}
+            bwd_mb = nb(t["q"], t["k"], t["v"], t["sinks"], o, l, t["dout"], dq, dk, dv, ds)
+            # full-causal 60k calls take ~40 ms (forward) and ~100 ms (backward)
+            n = 1 if (window == 0 and w.T > 60000) else iters
+            fns = {"fwd": f}
+            fns.update({"fwd:" + kn: (lambda kn=kn: f(kn)) for kn in FWD_KERNEL_NAMES})
+            ms = time_calls(torch, stream, fns, n, rounds=4, warm=1)
+            f()  # the backward reads the saved out / lse of sink_attn_fwd
+            ms.update(time_calls(torch, stream, {"bwd": b}, n, rounds=2, warm=1))
+            for name, tm in ms.items():
+                pas = name.split(":")[0]  # "fwd" or "bwd"
+                flops = (4 if pas == "fwd" else 10) * D * p
+                mb = fwd_mb if pas == "fwd" else bwd_mb
+                r = {"ms": tm, "tflops": flops / tm / 1e9, "pct_of_peak": 100.0 * flops / tm / 1e9 / peak,
+                     "min_bytes": mb, "GBps": mb / tm / 1e6, "hbm_frac": mb / tm / 1e6 / hbm}
                 if ":" in name:
                     lay.setdefault("fwd_kernels", {})[name.split(":")[1]] = r
                 else:
