@@ -104,13 +104,15 @@ struct FwdTile {
   int n_tiles; // 128-key K/V tiles to load
 };
 
+// Work unit `idx` (0 .. units x Hkv - 1; a CTA's blockIdx.x in the
+// non-persistent kernels).
 template <int kTiles>
-__device__ __forceinline__ FwdTile fwd_tile(const Geometry& geo) {
+__device__ __forceinline__ FwdTile fwd_tile(const Geometry& geo, int idx) {
   FwdTile w;
-  w.g = blockIdx.x % geo.Hkv;
+  w.g = idx % geo.Hkv;
   // Later tiles see more keys under a causal mask: hand them out first.
   const int units = (geo.num_qblocks + kTiles - 1) / kTiles;
-  const int u = units - 1 - static_cast<int>(blockIdx.x / geo.Hkv);
+  const int u = units - 1 - idx / geo.Hkv;
   w.t0 = (u * kTiles) << geo.P_log2;
   // first_key is non-decreasing in t: the first row has the smallest first
   // key, the last valid token the largest key.
@@ -205,7 +207,7 @@ __global__ void __launch_bounds__(kFwdThreads, 2)
   volatile int* abort = &ctl->abort;
   const int warp = threadIdx.x >> 5;
   const Geometry& geo = p.geo;
-  const FwdTile w = fwd_tile<kTiles>(geo);
+  const FwdTile w = fwd_tile<kTiles>(geo, static_cast<int>(blockIdx.x));
 
   if (threadIdx.x == 0) {
     mbar_init(&ctl->q_full, 1);
