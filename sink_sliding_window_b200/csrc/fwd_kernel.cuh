@@ -3,12 +3,13 @@
 //
 // Query tile: (128 / G) consecutive tokens x the G query heads of one
 // key/value head g, i.e. 128 MMA rows, row r <-> (token t0 + r / G, head
-// g*G + r % G).  In the one-tile mode (kTiles = 1) a CTA owns one tile.  Because q is [T][Hq][D], the G heads
-// of a group are contiguous and a single 3-D TMA box {64, G, 128/G} lands the
-// tile in exactly this row order.  Every key/value tile that is loaded serves
-// all G heads of the group.
+// g*G + r % G).  Because q is [T][Hq][D], the G heads of a group are
+// contiguous and a single 3-D TMA box {64, G, 128/G} lands the tile in
+// exactly this row order.  Every key/value tile that is loaded serves all G
+// heads of the group.
 //
-// Keys are consumed in steps of 64 ("halves" of a 128-key K/V tile):
+// One-tile mode (kTiles = 1): a CTA owns one query tile.  Keys are consumed
+// in steps of 64 ("halves" of a 128-key K/V tile):
 //   S_h = Q K_h^T          tcgen05.mma, bf16 in, fp32 in TMEM (64 columns),
 //                          into S/P buffer h % 2
 //   softmax (1 thread = 1 row, the row lives in that thread's TMEM lane):
@@ -25,9 +26,9 @@
 // (the sink is counted once, in warpgroup 0's seed).  While one warpgroup
 // waits for its next S, the other works on its own step; with two CTAs per
 // SM, four softmax warps share each SM sub-partition's exp2 unit.  A
-// warpgroup may rescale its
-// O_b without waiting for an MMA: the commit that announced S_h came after
-// the previous PV into O_b (tcgen05 MMAs of one thread execute in order).
+// warpgroup may rescale its O_b without waiting for an MMA: the commit that
+// announced S_h came after the previous PV into O_b (tcgen05 MMAs of one
+// thread execute in order).
 // Tiles outside the causal / window / document range are never visited; only
 // the edge steps apply an element mask.
 //

@@ -175,16 +175,19 @@ def fwd(q, k, v, sinks, cu_seqlens=None, window=0, scale=None, *, batch=None, ma
     return out, lse
 
 
-def fwd_pair(q, k, v, sinks, cu_seqlens=None, window=0, scale=None, **kw):
-    """sink_attn_fwd_pair: the forward on CTA pairs (tcgen05 M = 256)."""
-    dims, T, Hq, Hkv, D = _geometry(q, k, cu_seqlens, kw.get("batch"), kw.get("max_seqlen"))
-    out = kw.get("out")
-    lse = kw.get("lse")
-    out = torch.empty_like(q) if out is None else out
-    lse = torch.empty((Hq, T), dtype=torch.float32, device=q.device) if lse is None else lse
+def fwd_pair(q, k, v, sinks, cu_seqlens=None, window=0, scale=None, *, batch=None, max_seqlen=None, out=None,
+             lse=None, stream=None):
+    """sink_attn_fwd_pair: the forward on CTA pairs (tcgen05 M = 256);
+    arguments and results as fwd()."""
+    dims, T, Hq, Hkv, D = _geometry(q, k, cu_seqlens, batch, max_seqlen)
+    if scale is None:
+        scale = D ** -0.5
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((Hq, T), dtype=torch.float32, device=q.device)
     st = load().sink_attn_fwd_pair(ctypes.byref(dims), _ptr(q), _ptr(k), _ptr(v), _ptr(sinks), _ptr(cu_seqlens),
-                                   int(window), float(D ** -0.5 if scale is None else scale), _ptr(out), _ptr(lse),
-                                   _stream_handle(kw.get("stream")))
+                                   int(window), float(scale), _ptr(out), _ptr(lse), _stream_handle(stream))
     if st != 0:
         raise SinkAttnError(st, "sink_attn_fwd_pair")
     return out, lse
