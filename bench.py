@@ -179,16 +179,26 @@ def read_peaks():
 
 
 # Sources the backward main kernel is compiled from (its measured DRAM
-# traffic is reported only while these are unchanged).
+# traffic is reported only while their code is unchanged).
 BWD_MAIN_SOURCES = ("bwd_kernels.cuh", "common.cuh", "ptx.cuh", "tmem_io.cuh", "tma_host.cuh")
 
 
+def _code_only(text):
+    """C/C++ source without its comments and blank lines (string literals in
+    these headers hold no comment markers)."""
+    import re
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    return "\n".join(line.rstrip() for line in text.splitlines() if line.strip())
+
+
 def kernel_source_hash():
+    """Hash of the code (comments excluded) of BWD_MAIN_SOURCES."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "sink_sliding_window_b200", "csrc")
     for n in BWD_MAIN_SOURCES:
-        with open(os.path.join(csrc, n), "rb") as f:
-            h.update(n.encode() + f.read())
+        with open(os.path.join(csrc, n), encoding="utf-8") as f:
+            h.update(n.encode() + _code_only(f.read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -75,7 +75,8 @@ __device__ __forceinline__ bool mbar_wait_cl(uint64_t* bar, uint32_t parity, vol
 
 // 3-D tiled TMA load into this CTA's shared memory whose completion (the
 // box's bytes) is signalled on a barrier of either CTA of the pair, given by
-// its shared::cluster address.  No multicast: each CTA loads its own boxes.
+// its shared::cluster address.  Each CTA loads its own boxes; no load is
+// shared between the CTAs.
 // x keeps the 16-byte alignment TMA needs (callers pass 0 or 32 bf16).
 __device__ __forceinline__ void tma_load_3d_pair(void* smem_dst, const CUtensorMap* map, uint32_t bar_cluster, int x,
                                                  int y, int z) {

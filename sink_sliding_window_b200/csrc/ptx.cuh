@@ -1,5 +1,5 @@
 // Thin inline-PTX wrappers for the sm_100a features the kernels use:
-// mbarriers with bounded waits, TMA tensor loads (no multicast), and the
+// mbarriers with bounded waits, TMA tensor loads (each CTA loads its own boxes), and the
 // tcgen05 tensor-core path (TMEM allocation, MMA, commit, fences).
 #pragma once
 #include <cuda.h>
