@@ -68,7 +68,7 @@ def test_lengths_and_windows(ops, S, window):
     _whole(ops, w, a, f"S={S} W={window}")
 
 
-@pytest.mark.parametrize("G", [1, 2, 4, 8, 16])
+@pytest.mark.parametrize("G", [1, 2, 4, 8, 16, 32, 64, 128])
 def test_gqa_ratios(ops, G):
     w, a = _small(400, G * 2, 2, [0, 37, 38, 400], 100, seed=G + 50)
     _whole(ops, w, a, f"G={G}")

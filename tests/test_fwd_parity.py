@@ -73,7 +73,7 @@ def test_lengths_and_windows(ops, S, window):
     _whole_check(ops, w, a, f"S={S} W={window}")
 
 
-@pytest.mark.parametrize("G", [1, 2, 4, 8, 16, 32])
+@pytest.mark.parametrize("G", [1, 2, 4, 8, 16, 32, 64, 128])
 def test_gqa_ratios(ops, G):
     Hkv = 2
     w, a = _small(400, G * Hkv, Hkv, [0, 37, 38, 400], 100, seed=G)
