@@ -32,6 +32,27 @@ def test_exports_every_declared_symbol(L):
     assert set(ops.EXPORTS) <= set(names)
 
 
+def test_header_is_c_and_links(L, tmp_path):
+    """include/sink_attn.h is plain C (C99, pedantic, warnings as errors),
+    and a C program that takes the address of every declared function links
+    against the built library."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("gcc not available")
+    names = declared_functions()
+    body = "\n".join(f"  (void)&{n};" for n in names)
+    src = tmp_path / "abi_check.c"
+    src.write_text(f'#include "sink_attn.h"\nint main(void) {{\n{body}\n  return 0;\n}}\n')
+    lib_dir = os.path.dirname(ops.lib_path())
+    cmd = [gcc, "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", "-I", os.path.join(ROOT, "include"),
+           str(src), "-o", str(tmp_path / "abi_check"), "-L", lib_dir, "-l:" + os.path.basename(ops.lib_path()),
+           f"-Wl,-rpath,{lib_dir}"]
+    r = subprocess.run(cmd, capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+
+
 def test_status_strings(L):
     for code in range(8):
         s = ops.status_string(code)
