@@ -247,7 +247,11 @@ struct BwdCtl {
   uint64_t s_full[2];
   uint64_t dp_full;
   uint64_t p_full;
-  uint64_t dq_full;
+  // dQ_i ready in TMEM, one barrier per tile parity: tile i+2's dQ can only
+  // be committed after the dQ warps released tile i's TMEM (dq_empty), so a
+  // barrier never runs two phases ahead of the dQ warps' parity wait, however
+  // late the dQ warps are.
+  uint64_t dq_full[2];
   uint64_t dq_empty;
   uint64_t kd_full;
   uint64_t dq_sync;       // the four dQ warps (128 threads)
@@ -379,7 +383,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     mbar_init(&ctl->s_full[1], 1);
     mbar_init(&ctl->dp_full, 1);
     mbar_init(&ctl->p_full, 256);
-    mbar_init(&ctl->dq_full, 1);
+    mbar_init(&ctl->dq_full[0], 1);
+    mbar_init(&ctl->dq_full[1], 1);
     mbar_init(&ctl->dq_empty, 128);
     mbar_init(&ctl->kd_full, 1);
     mbar_init(&ctl->dq_sync, 128);
@@ -490,7 +495,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         for (int kk = 0; kk < kBlockN / 16; ++kk)
           mma_ss(tSb + 64, make_sdesc_sw128(ds_addr + kk * 2048, 16384, 1024),
                  make_sdesc_sw128(k_addr + kk * 2048, kTileBytes, 1024), idesc_dq, kk > 0);
-        tc_commit(&ctl->dq_full);
+        tc_commit(&ctl->dq_full[i & 1]);
         tc_commit(&ctl->qdo_empty[st]);
         if (i + 1 < w.nq) {
           // dP^T_{i+1} (dS_i in the dP region was consumed by dK above)
@@ -639,7 +644,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     uint32_t sync_phase = 0;
     bool ok = true;
     for (int i = 0; i < w.nq; ++i) {
-      ok = warp_all(mbar_wait(&ctl->dq_full, i & 1, abort, &g_device_error, kDevErrTimeoutBwd));
+      ok = warp_all(mbar_wait(&ctl->dq_full[i & 1], (i >> 1) & 1, abort, &g_device_error, kDevErrTimeoutBwd));
       if (!ok) break;
       tc_fence_after();
       uint32_t d[kHeadDim];
