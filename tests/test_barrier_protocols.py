@@ -1,0 +1,253 @@
+"""Models of the mbarrier protocols of the backward main kernel and of the
+two-tile forward, run under random interleavings (CPU only).
+
+Each kernel role (TMA producer, MMA issuer, softmax or P/dS warps, dQ warps)
+is a generator that waits on and arrives at barriers in the order the kernel
+does; tcgen05 MMAs and their commits complete in issue order on a separate
+"tensor core" queue, TMA loads complete in any order.  A parity wait on
+phase k is only unambiguous while the barrier has completed at most k + 1
+phases: the model asserts that at every check, and that every schedule runs
+to completion (no deadlock).  The models follow the kernels' barrier use,
+not their arithmetic; they must be kept in step with the kernels by hand.
+"""
+import random
+
+import pytest
+
+
+class Ambiguous(AssertionError):
+    pass
+
+
+class Bar:
+    def __init__(self, name, count):
+        self.name, self.count, self.arr, self.done = name, count, 0, 0
+
+    def arrive(self, n=1):
+        self.arr += n
+        assert self.arr <= self.count, f"{self.name}: too many arrivals"
+        if self.arr == self.count:
+            self.arr = 0
+            self.done += 1
+
+    def test(self, k):
+        """Parity wait for phase k: true once phase k completed; raises if
+        the barrier is two phases ahead (a parity wait would read it as
+        incomplete)."""
+        if self.done >= k + 2:
+            raise Ambiguous(f"{self.name}: waiting for phase {k}, {self.done} phases done")
+        return self.done > k
+
+
+def _run(agents, tc_queue, tma, rng, limit=200000):
+    """Random scheduler: steps agents, the in-order tensor-core queue and the
+    unordered TMA completions until every agent finished."""
+    alive = list(range(len(agents)))
+    idle = 0
+    for _ in range(limit):
+        if not alive and not tc_queue and not tma:
+            return
+        c = rng.random()
+        progressed = False
+        if c < 0.2 and tma:
+            tma.pop(rng.randrange(len(tma))).arrive()
+            progressed = True
+        elif c < 0.4 and tc_queue:
+            op = tc_queue.pop(0)
+            if op is not None:
+                op()
+            progressed = True
+        elif alive:
+            i = rng.choice(alive)
+            try:
+                progressed = next(agents[i]) != "blocked"
+            except StopIteration:
+                alive.remove(i)
+                progressed = True
+        idle = 0 if progressed else idle + 1
+        if idle > 5000 and not tc_queue and not tma:
+            raise AssertionError(f"deadlock: agents {alive} blocked")
+    raise AssertionError("schedule did not finish")
+
+
+def _wait(bar, k):
+    while not bar.test(k):
+        yield "blocked"
+
+
+# ----------------------------------------------------------- backward main
+def backward_model(nq, stages, split_dq_full, dq_delay, rng):
+    """One CTA of the backward main kernel over nq query tiles.
+    split_dq_full: one dq_full barrier per tile parity (the kernel's scheme)
+    or a single one; dq_delay: extra steps the dQ warps spend per tile."""
+    B = {}
+
+    def bar(name, count=1):
+        return B.setdefault(name, Bar(name, count))
+
+    for s in range(stages):
+        bar(("qdo_full", s))
+        bar(("qdo_empty", s))
+    for b in range(2):
+        bar(("s_full", b))
+        bar(("dq_full", b))
+    bar("dp_full")
+    bar("p_full")
+    bar("dq_empty")
+    bar("kd_full")
+    tc, tma = [], []
+
+    def dq_full(i):
+        return bar(("dq_full", i & 1)) if split_dq_full else bar(("dq_full", 0))
+
+    def dq_phase(i):
+        return (i >> 1) if split_dq_full else i
+
+    def producer():
+        for i in range(nq):
+            s = i % stages
+            if i >= stages:
+                yield from _wait(bar(("qdo_empty", s)), i // stages - 1)
+            tma.append(bar(("qdo_full", s)))
+            yield "ok"
+
+    def mma():
+        def wait_q(i):
+            return _wait(bar(("qdo_full", i % stages)), i // stages)
+        yield from wait_q(0)
+        tc.append(lambda: bar(("s_full", 0)).arrive())
+        tc.append(lambda: bar("dp_full").arrive())
+        if nq > 1:
+            yield from wait_q(1)
+            tc.append(lambda: bar(("s_full", 1)).arrive())
+        for i in range(nq):
+            yield from _wait(bar("p_full"), i)
+            st = i % stages
+            tc.append(None)  # dV, dK, dQ MMAs
+            tc.append(lambda i=i: dq_full(i).arrive())
+            tc.append(lambda st=st: bar(("qdo_empty", st)).arrive())
+            if i + 1 < nq:
+                yield from wait_q(i + 1)
+                tc.append(lambda: bar("dp_full").arrive())
+            if i + 2 < nq:
+                yield from _wait(bar("dq_empty"), i)
+                yield from wait_q(i + 2)
+                tc.append(lambda i=i: bar(("s_full", i & 1)).arrive())
+        tc.append(lambda: bar("kd_full").arrive())
+
+    def pds():
+        for i in range(nq):
+            yield from _wait(bar(("qdo_full", i % stages)), i // stages)
+            yield from _wait(bar(("s_full", i & 1)), i >> 1)
+            yield "ok"  # P phase
+            yield from _wait(bar("dp_full"), i)
+            yield "ok"  # dS phase
+            bar("p_full").arrive()
+        yield from _wait(bar("kd_full"), 0)
+
+    def dq():
+        for i in range(nq):
+            yield from _wait(dq_full(i), dq_phase(i))
+            bar("dq_empty").arrive()
+            for _ in range(dq_delay):
+                yield "ok"
+
+    return [producer(), mma(), pds(), dq()], tc, tma
+
+
+@pytest.mark.parametrize("nq", [1, 2, 3, 5, 17])
+@pytest.mark.parametrize("dq_delay", [0, 3, 40])
+def test_backward_protocol(nq, dq_delay):
+    """The kernel's scheme (dq_full per tile parity) is unambiguous and
+    deadlock-free however slow the dQ warps are."""
+    rng = random.Random(nq * 1000 + dq_delay)
+    for _ in range(150):
+        agents, tc, tma = backward_model(nq, 3, True, dq_delay, rng)
+        _run(agents, tc, tma, rng)
+
+
+def test_backward_single_dq_full_is_ambiguous_when_dq_is_slow():
+    """The model catches the race of a single dq_full barrier: once the dQ
+    warps release tile i's TMEM, the MMA warp can complete the dQ of tiles
+    i+1 and i+2 before a slow dQ warp waits for tile i+1."""
+    rng = random.Random(7)
+    caught = False
+    for _ in range(300):
+        agents, tc, tma = backward_model(8, 3, False, 40, rng)
+        try:
+            _run(agents, tc, tma, rng)
+        except Ambiguous:
+            caught = True
+            break
+    assert caught
+
+
+# ------------------------------------------------------- two-tile forward
+def forward_two_tile_model(n_half, stages, rng):
+    """One CTA of the two-tile forward over n_half 64-key steps (two steps
+    per 128-key K/V tile, stages K/V tile buffers)."""
+    B = {}
+
+    def bar(name, count=1):
+        return B.setdefault(name, Bar(name, count))
+
+    bar("q_full")
+    for s in range(stages):
+        bar(("k_full", s))
+        bar(("v_full", s))
+        bar(("kv_empty", s))
+    for b in range(2):
+        bar(("s_full", b))
+        bar(("p_full", b))
+    bar("o_full")
+    tc, tma = [], []
+    n_tiles = (n_half + 1) // 2
+
+    def producer():
+        tma.append(bar("q_full"))
+        for j in range(n_tiles):
+            s = j % stages
+            if j >= stages:
+                yield from _wait(bar(("kv_empty", s)), j // stages - 1)
+            tma.append(bar(("k_full", s)))
+            tma.append(bar(("v_full", s)))
+            yield "ok"
+
+    def mma():
+        yield from _wait(bar("q_full"), 0)
+        yield from _wait(bar(("k_full", 0)), 0)
+        for b in range(2):
+            tc.append(lambda b=b: bar(("s_full", b)).arrive())
+        for h in range(n_half):
+            j = h >> 1
+            s = j % stages
+            hn = h + 1
+            jn = hn >> 1
+            yield from _wait(bar(("v_full", s)), j // stages)
+            if hn < n_half:
+                yield from _wait(bar(("k_full", jn % stages)), jn // stages)
+            for b in range(2):
+                yield from _wait(bar(("p_full", b)), h)
+                tc.append(None)  # PV_b(h)
+                if hn < n_half:
+                    tc.append(lambda b=b: bar(("s_full", b)).arrive())
+            if (h & 1) == 1 or h == n_half - 1:
+                tc.append(lambda s=s: bar(("kv_empty", s)).arrive())
+        tc.append(lambda: bar("o_full").arrive())
+
+    def softmax(b):
+        for h in range(n_half):
+            yield from _wait(bar(("s_full", b)), h)
+            yield "ok"
+            bar(("p_full", b)).arrive()
+        yield from _wait(bar("o_full"), 0)
+
+    return [producer(), mma(), softmax(0), softmax(1)], tc, tma
+
+
+@pytest.mark.parametrize("n_half", [1, 2, 3, 4, 7, 20])
+def test_forward_two_tile_protocol(n_half):
+    rng = random.Random(n_half)
+    for _ in range(200):
+        agents, tc, tma = forward_two_tile_model(n_half, 2, rng)
+        _run(agents, tc, tma, rng)
