@@ -1,5 +1,6 @@
-"""Models of the mbarrier protocols of the backward main kernel and of the
-two-tile forward, run under random interleavings (CPU only).
+"""Models of the mbarrier protocols of the backward main kernel, the
+two-tile forward and the CTA-pair forward, run under random interleavings
+(CPU only).
 
 Each kernel role (TMA producer, MMA issuer, softmax or P/dS warps, dQ warps)
 is a generator that waits on and arrives at barriers in the order the kernel
@@ -7,7 +8,9 @@ does; tcgen05 MMAs and their commits complete in issue order on a separate
 "tensor core" queue, TMA loads complete in any order.  A parity wait on
 phase k is only unambiguous while the barrier has completed at most k + 1
 phases: the model asserts that at every check, and that every schedule runs
-to completion (no deadlock).  The models follow the kernels' barrier use,
+to completion (no deadlock).  Barriers that receive TMA bytes also count
+transactions, so the pair model checks that the peer CTA's bytes landing
+before the leader announced them cannot complete a phase early.  The models follow the kernels' barrier use,
 not their arithmetic; they must be kept in step with the kernels by hand.
 """
 import random
@@ -20,15 +23,27 @@ class Ambiguous(AssertionError):
 
 
 class Bar:
-    def __init__(self, name, count):
-        self.name, self.count, self.arr, self.done = name, count, 0, 0
+    """An mbarrier: a phase completes when its pending arrivals reach zero
+    and its transaction count (expect-tx adds, complete-tx subtracts; it may
+    go negative in between) is zero."""
 
-    def arrive(self, n=1):
-        self.arr += n
-        assert self.arr <= self.count, f"{self.name}: too many arrivals"
-        if self.arr == self.count:
+    def __init__(self, name, count):
+        self.name, self.count, self.arr, self.done, self.tx = name, count, 0, 0, 0
+
+    def _maybe_complete(self):
+        if self.arr == self.count and self.tx == 0:
             self.arr = 0
             self.done += 1
+
+    def arrive(self, n=1, expect_tx=0):
+        self.tx += expect_tx
+        self.arr += n
+        assert self.arr <= self.count, f"{self.name}: too many arrivals"
+        self._maybe_complete()
+
+    def complete_tx(self, nbytes):
+        self.tx -= nbytes
+        self._maybe_complete()
 
     def test(self, k):
         """Parity wait for phase k: true once phase k completed; raises if
@@ -50,7 +65,8 @@ def _run(agents, tc_queue, tma, rng, limit=200000):
         c = rng.random()
         progressed = False
         if c < 0.2 and tma:
-            tma.pop(rng.randrange(len(tma))).arrive()
+            t = tma.pop(rng.randrange(len(tma)))
+            t() if callable(t) else t.arrive()
             progressed = True
         elif c < 0.4 and tc_queue:
             op = tc_queue.pop(0)
@@ -250,4 +266,107 @@ def test_forward_two_tile_protocol(n_half):
     rng = random.Random(n_half)
     for _ in range(200):
         agents, tc, tma = forward_two_tile_model(n_half, 2, rng)
+        _run(agents, tc, tma, rng)
+
+
+# ----------------------------------------------------------- pair forward
+def forward_pair_model(n_half, stages, rng):
+    """A cluster of two CTAs of the pair forward over n_half 64-key steps.
+    The leader's q_full / k_full / v_full receive both CTAs' TMA bytes (each
+    CTA loads its half; the peer's bytes may land before the leader announced
+    them); the leader's p_full takes one arrival per softmax warp of either
+    CTA; s_full, kv_empty and o_full exist in both CTAs and the leader commits
+    to both.  Each K or V half is one transaction of HALF bytes."""
+    HALF = 4096
+    B = {}
+
+    def bar(name, count=1):
+        return B.setdefault(name, Bar(name, count))
+
+    for c in range(2):
+        for s in range(stages):
+            bar(("kv_empty", c, s))
+        for b in range(2):
+            bar(("s_full", c, b))
+        bar(("o_full", c))
+    bar("q_full")
+    for s in range(stages):
+        bar(("k_full", s))
+        bar(("v_full", s))
+    for b in range(2):
+        bar(("p_full", b), 8)
+    landed = {}  # (kind, step, cta) -> the CTA's half of the step is in its shared memory
+    tc, tma = [], []
+
+    def load(kind, key, cta, nbytes):
+        def land():
+            landed[(kind, key, cta)] = True
+            bar(kind if kind == "q_full" else (kind, key % stages)).complete_tx(nbytes)
+        return land
+
+    def producer(cta):
+        if cta == 0:
+            bar("q_full").arrive(expect_tx=2 * 16384)
+        tma.append(load("q_full", 0, cta, 16384))
+        for h in range(n_half):
+            s = h % stages
+            if h >= stages:
+                yield from _wait(bar(("kv_empty", cta, s)), h // stages - 1)
+            if cta == 0:
+                bar(("k_full", s)).arrive(expect_tx=2 * HALF)
+            tma.append(load("k_full", h, cta, HALF))
+            if cta == 0:
+                bar(("v_full", s)).arrive(expect_tx=2 * HALF)
+            tma.append(load("v_full", h, cta, HALF))
+            yield "ok"
+
+    def both(name):
+        def commit():
+            for c in range(2):
+                bar((name[0], c) + name[1:]).arrive()
+        return commit
+
+    def mma():
+        yield from _wait(bar("q_full"), 0)
+        assert landed.get(("q_full", 0, 0)) and landed.get(("q_full", 0, 1))
+        for h in range(min(2, n_half)):
+            yield from _wait(bar(("k_full", h)), 0)
+            assert landed.get(("k_full", h, 0)) and landed.get(("k_full", h, 1)), f"S({h}) before K landed"
+            tc.append(both(("s_full", h)))
+        for h in range(n_half):
+            b = h & 1
+            s = h % stages
+            yield from _wait(bar(("v_full", s)), h // stages)
+            assert landed.get(("v_full", h, 0)) and landed.get(("v_full", h, 1)), f"PV({h}) before V landed"
+            yield from _wait(bar(("p_full", b)), h >> 1)
+            tc.append(None)  # PV(h)
+            tc.append(both(("kv_empty", s)))
+            h2 = h + 2
+            if h2 < n_half:
+                yield from _wait(bar(("k_full", h2 % stages)), h2 // stages)
+                assert landed.get(("k_full", h2, 0)) and landed.get(("k_full", h2, 1)), f"S({h2}) before K landed"
+                tc.append(both(("s_full", b)))
+        tc.append(both(("o_full",)))
+
+    def softmax(cta, wg):
+        i = 0
+        for hs in range(wg, n_half, 2):
+            yield from _wait(bar(("s_full", cta, wg)), i)
+            yield "ok"
+            bar(("p_full", wg)).arrive(4)  # one arrival per warp of the warpgroup
+            i += 1
+        yield from _wait(bar(("o_full", cta)), 0)
+
+    agents = [producer(0), producer(1), mma()] + [softmax(c, w) for c in range(2) for w in range(2)]
+    return agents, tc, tma
+
+
+@pytest.mark.parametrize("n_half", [1, 2, 3, 5, 9, 20])
+def test_forward_pair_protocol(n_half):
+    """Both CTAs' halves of Q, K and V have landed whenever the leader's
+    barrier says so (the peer's bytes may arrive before the leader's
+    expect-tx), parity waits stay unambiguous, no schedule deadlocks."""
+    rng = random.Random(100 + n_half)
+    for _ in range(200):
+        agents, tc, tma = forward_pair_model(n_half, 4, rng)
         _run(agents, tc, tma, rng)
