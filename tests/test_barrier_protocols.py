@@ -1,6 +1,6 @@
-"""Models of the mbarrier protocols of the backward main kernel, the
-two-tile forward and the CTA-pair forward, run under random interleavings
-(CPU only).
+"""Models of the mbarrier protocols of the backward main kernel and of the
+forward kernels (two tiles per CTA, one tile per CTA, CTA pairs), run under
+random interleavings (CPU only).
 
 Each kernel role (TMA producer, MMA issuer, softmax or P/dS warps, dQ warps)
 is a generator that waits on and arrives at barriers in the order the kernel
@@ -369,4 +369,74 @@ def test_forward_pair_protocol(n_half):
     rng = random.Random(100 + n_half)
     for _ in range(200):
         agents, tc, tma = forward_pair_model(n_half, 4, rng)
+        _run(agents, tc, tma, rng)
+
+
+# -------------------------------------------------------- one-tile forward
+def forward_one_tile_model(n_half, stages, rng):
+    """One CTA of the one-tile forward: the tile's 64-key steps alternate
+    between the two softmax warpgroups (step h to warpgroup h % 2)."""
+    B = {}
+
+    def bar(name, count=1):
+        return B.setdefault(name, Bar(name, count))
+
+    bar("q_full")
+    for s in range(stages):
+        bar(("k_full", s))
+        bar(("v_full", s))
+        bar(("kv_empty", s))
+    for b in range(2):
+        bar(("s_full", b))
+        bar(("p_full", b))
+    bar("o_full")
+    tc, tma = [], []
+    n_tiles = (n_half + 1) // 2
+
+    def producer():
+        tma.append(bar("q_full"))
+        for j in range(n_tiles):
+            s = j % stages
+            if j >= stages:
+                yield from _wait(bar(("kv_empty", s)), j // stages - 1)
+            tma.append(bar(("k_full", s)))
+            tma.append(bar(("v_full", s)))
+            yield "ok"
+
+    def mma():
+        yield from _wait(bar("q_full"), 0)
+        for h in range(min(2, n_half)):
+            yield from _wait(bar(("k_full", 0)), 0)
+            tc.append(lambda h=h: bar(("s_full", h)).arrive())
+        for h in range(n_half):
+            b = h & 1
+            j = h >> 1
+            s = j % stages
+            yield from _wait(bar(("v_full", s)), j // stages)
+            yield from _wait(bar(("p_full", b)), h >> 1)
+            tc.append(None)  # PV(h)
+            if b == 1 or h == n_half - 1:
+                tc.append(lambda s=s: bar(("kv_empty", s)).arrive())
+            h2 = h + 2
+            if h2 < n_half:
+                j2 = h2 >> 1
+                yield from _wait(bar(("k_full", j2 % stages)), j2 // stages)
+                tc.append(lambda b=b: bar(("s_full", b)).arrive())
+        tc.append(lambda: bar("o_full").arrive())
+
+    def softmax(b):
+        for i, _ in enumerate(range(b, n_half, 2)):
+            yield from _wait(bar(("s_full", b)), i)
+            yield "ok"
+            bar(("p_full", b)).arrive()
+        yield from _wait(bar("o_full"), 0)
+
+    return [producer(), mma(), softmax(0), softmax(1)], tc, tma
+
+
+@pytest.mark.parametrize("n_half", [1, 2, 3, 4, 7, 20])
+def test_forward_one_tile_protocol(n_half):
+    rng = random.Random(300 + n_half)
+    for _ in range(200):
+        agents, tc, tma = forward_one_tile_model(n_half, 2, rng)
         _run(agents, tc, tma, rng)
