@@ -1,6 +1,7 @@
-"""Models of the mbarrier protocols of the backward main kernel and of the
-forward kernels (two tiles per CTA, one tile per CTA, CTA pairs), run under
-random interleavings (CPU only).
+"""Models of the mbarrier protocols of the backward main kernel, the forward
+kernels (two tiles per CTA, one tile per CTA, CTA pairs) and the decode
+kernel (bf16 cache, e4m3 cache, e4m3 cache with the FP8 PV product), run
+under random interleavings (CPU only).
 
 Each kernel role (TMA producer, MMA issuer, softmax or P/dS warps, dQ warps)
 is a generator that waits on and arrives at barriers in the order the kernel
@@ -439,4 +440,116 @@ def test_forward_one_tile_protocol(n_half):
     rng = random.Random(300 + n_half)
     for _ in range(200):
         agents, tc, tma = forward_one_tile_model(n_half, 2, rng)
+        _run(agents, tc, tma, rng)
+
+
+# ------------------------------------------------------------------ decode
+def decode_model(n, stages, mode, rng):
+    """One CTA of the decode kernel over n 128-slot tiles.  mode 0: bf16
+    cache; 1: e4m3 cache widened by the converter warps (K into TMEM, V into
+    two fp16 tiles); 2: e4m3 cache with the FP8 PV product (K widened, V read
+    as loaded).  Groups of 128 threads arrive together."""
+    f8, pv8 = mode >= 1, mode == 2
+    B = {}
+
+    def bar(name, count=1):
+        return B.setdefault(name, Bar(name, count))
+
+    bar("q_full")
+    bar("q_conv")
+    for s in range(stages):
+        bar(("k_full", s))
+        bar(("k_empty", s))
+        bar(("v_full", s))
+        bar(("v_empty", s))
+    for b in range(2):
+        bar(("s_full", b))
+        bar(("s_free", b))
+        bar(("kt_full", b))
+        bar(("pv_done", b))
+        bar(("v_ready", b))
+    bar("p_full")
+    bar("o_full")
+    tc, tma = [], []
+
+    def producer():
+        tma.append(bar("q_full"))
+        for i in range(n):
+            s = i % stages
+            if i >= stages:
+                yield from _wait(bar(("k_empty", s)), i // stages - 1)
+            tma.append(bar(("k_full", s)))
+            if i >= stages:
+                yield from _wait(bar(("v_empty", s)), i // stages - 1)
+            tma.append(bar(("v_full", s)))
+            yield "ok"
+
+    def converter():
+        yield from _wait(bar("q_full"), 0)
+        bar("q_conv").arrive()
+        for i in range(n):
+            b, s = i & 1, i % stages
+            if i >= 2:
+                yield from _wait(bar(("s_full", b)), (i - 2) >> 1)
+            yield from _wait(bar(("k_full", s)), i // stages)
+            bar(("k_empty", s)).arrive()
+            bar(("kt_full", b)).arrive()
+            if pv8:
+                continue
+            if i >= 2:
+                yield from _wait(bar(("pv_done", i & 1)), (i - 2) >> 1)
+            yield from _wait(bar(("v_full", s)), i // stages)
+            bar(("v_empty", s)).arrive()
+            bar(("v_ready", i & 1)).arrive()
+
+    def mma():
+        yield from _wait(bar("q_conv" if f8 else "q_full"), 0)
+        for i in range(n + 1):
+            if i < n:
+                b, s = i & 1, i % stages
+                if i >= 2:
+                    yield from _wait(bar(("s_free", b)), (i >> 1) - 1)
+                if f8:
+                    yield from _wait(bar(("kt_full", b)), i >> 1)
+                else:
+                    yield from _wait(bar(("k_full", s)), i // stages)
+                tc.append(lambda b=b: bar(("s_full", b)).arrive())
+                if not f8:
+                    tc.append(lambda s=s: bar(("k_empty", s)).arrive())
+            if i >= 1:
+                j = i - 1
+                sj = j % stages
+                yield from _wait(bar("p_full"), j)
+                if f8 and not pv8:
+                    yield from _wait(bar(("v_ready", j & 1)), j >> 1)
+                else:
+                    yield from _wait(bar(("v_full", sj)), j // stages)
+                tc.append(lambda j=j: bar(("pv_done", j & 1)).arrive())
+                if not f8 or pv8:
+                    tc.append(lambda sj=sj: bar(("v_empty", sj)).arrive())
+        tc.append(lambda: bar("o_full").arrive())
+
+    def softmax():
+        for i in range(n):
+            b = i & 1
+            yield from _wait(bar(("s_full", b)), i >> 1)
+            bar(("s_free", b)).arrive()
+            yield "ok"
+            if i > 0:
+                yield from _wait(bar(("pv_done", (i - 1) & 1)), (i - 1) >> 1)
+            if (not f8 or pv8) and rng.random() < 0.5:  # a tile with empty slots: zero their V rows
+                yield from _wait(bar(("v_full", i % stages)), i // stages)
+            bar("p_full").arrive()
+        yield from _wait(bar("o_full"), 0)
+
+    agents = [producer(), mma(), softmax()] + ([converter()] if f8 else [])
+    return agents, tc, tma
+
+
+@pytest.mark.parametrize("mode", [0, 1, 2])
+@pytest.mark.parametrize("n", [1, 2, 3, 6, 13])
+def test_decode_protocol(mode, n):
+    rng = random.Random(500 + 10 * mode + n)
+    for _ in range(150):
+        agents, tc, tma = decode_model(n, 2, mode, rng)
         _run(agents, tc, tma, rng)
