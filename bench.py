@@ -315,7 +315,7 @@ def measure_layers(torch, ops, stream, q, k, v, sinks, dout, outs, grads, ws, it
     the launching stream, the forward kernels taken in turn): TFLOP/s on the
     counted pairs, and GB/s of the layer's minimum DRAM bytes (every input
     read once, every output written once) against the measured HBM peak; the
-    window-128 layers are judged on the latter.  "fwd" is sink_attn_fwd (the
+    window-128 layers are rated by the latter.  "fwd" is sink_attn_fwd (the
     kernel it picks is named), "fwd_kernels" each forward kernel through
     sink_attn_fwd_with.  q, dout, out and dq (134 MB each) exceed the 126 MB
     L2, so no flush between calls."""

@@ -67,7 +67,7 @@ typedef enum {
     SINK_ATTN_ERR_NULL = 1,          /* a required pointer is NULL */
     SINK_ATTN_ERR_SHAPE = 2,         /* inconsistent or negative sizes */
     SINK_ATTN_ERR_ALIGN = 3,         /* a tensor is not 16-byte aligned */
-    SINK_ATTN_ERR_UNSUPPORTED = 4,   /* valid, but outside what this build implements */
+    SINK_ATTN_ERR_UNSUPPORTED = 4,   /* valid, but outside what this library implements */
     SINK_ATTN_ERR_CUDA = 5,          /* a CUDA runtime/driver call failed */
     SINK_ATTN_ERR_DEVICE_TIMEOUT = 6,/* a kernel gave up on a wait (see sink_attn_last_device_error) */
     SINK_ATTN_ERR_WORKSPACE = 7      /* workspace missing or smaller than sink_attn_bwd_workspace_size() */
