@@ -157,6 +157,8 @@ def fwd(q, k, v, sinks, cu_seqlens=None, window=0, scale=None, *, batch=None, ma
     library's forward kernels ("one_tile", "two_tiles", "pair").  q [T,Hq,D]
     (or [B,S,Hq,D]), k/v [T,Hkv,D] bf16 CUDA; sinks [Hq] fp32; cu_seqlens
     int32 [B+1] CUDA or None.  Returns (out like q, lse [Hq, T] fp32)."""
+    if kernel not in FWD_KERNELS:
+        raise ValueError(f"unknown forward kernel {kernel!r}; expected one of {sorted(FWD_KERNELS)}")
     dims, T, Hq, Hkv, D = _geometry(q, k, cu_seqlens, batch, max_seqlen)
     if scale is None:
         scale = D ** -0.5

@@ -125,6 +125,11 @@ def test_fwd_with_rejects_unknown_kernel(L):
                                 None) == 1
 
 
+def test_fwd_binding_rejects_unknown_kernel_name():
+    with pytest.raises(ValueError):
+        ops.fwd(None, None, None, None, kernel="bogus")
+
+
 def test_fwd_kernel_for(L):
     for window in (0, 1, 128, 4096):
         assert L.sink_attn_fwd_kernel_for(ctypes.byref(dims()), window) in (1, 2, 3)
